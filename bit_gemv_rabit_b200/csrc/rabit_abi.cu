@@ -1,0 +1,190 @@
+// rabit_abi.cu -- the extern "C" boundary of librabit (declared in include/rabit.h).
+//
+// Each entry point validates every argument on the host before anything is enqueued
+// (pure argument checks first, then the device checks), then calls one launcher.  Nothing
+// here computes any part of the layer: all arithmetic runs in the CUDA kernels.
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "rabit.h"
+#include "rabit_kernels.h"
+
+namespace {
+
+// Per-device fault word: bit set by a kernel whose bounded wait expired.
+__device__ uint32_t g_fault_word = 0;
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    int state;  // 0 unknown, 1 ok (sm_100), 2 wrong arch
+    int num_sms;
+    uint32_t *fault_ptr;
+};
+DeviceInfo g_devices[kMaxDevices];
+
+int cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return RABIT_ERR_CUDA;
+}
+
+bool env_flag(const char *name) {
+    const char *v = std::getenv(name);
+    return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+// Validates the current device; fills ctx.  Returns RABIT_OK or an error status.
+int device_ctx(void *stream, rabit::LaunchCtx &ctx, uint32_t **fault_ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return RABIT_ERR_ARCH;
+    DeviceInfo &info = g_devices[dev];
+    if (info.state == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        void *fp = nullptr;
+        if (major == 10 && minor == 0) {
+            if ((e = cudaGetSymbolAddress(&fp, g_fault_word)) != cudaSuccess) return cuda_fail(e);
+        }
+        info.num_sms = sms;
+        info.fault_ptr = static_cast<uint32_t *>(fp);
+        info.state = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    if (info.state != 1 || env_flag("RABIT_TEST_FORCE_ARCH_MISMATCH")) return RABIT_ERR_ARCH;
+    ctx.stream = static_cast<cudaStream_t>(stream);
+    ctx.num_sms = info.num_sms;
+    ctx.pdl = !(std::getenv("RABIT_PDL") && std::strcmp(std::getenv("RABIT_PDL"), "0") == 0);
+    if (fault_ptr) *fault_ptr = info.fault_ptr;
+    return RABIT_OK;
+}
+
+bool aligned(const void *p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+// Bound on every device-side wait: 2 s, far above any real wait, unless overridden.
+uint64_t wait_timeout_ns() {
+    uint64_t timeout_ns = 2000000000ull;
+    if (const char *t = std::getenv("RABIT_WAIT_TIMEOUT_MS")) {
+        const long long ms = std::atoll(t);
+        if (ms > 0) timeout_ns = static_cast<uint64_t>(ms) * 1000000ull;
+    }
+    return timeout_ns;
+}
+
+int finish_launch(cudaError_t e) {
+    if (e != cudaSuccess) return cuda_fail(e);
+    return RABIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rabit_packed_words(int N, int K, int P) {
+    if (N < 1 || K < 1 || P < 1) return 0;
+    const size_t group = P == 2 ? 2 : (P == 1 ? 1 : 4);
+    return static_cast<size_t>(N) * static_cast<size_t>(rabit::padded_cols(K) / 32) * group;
+}
+
+size_t rabit_gemm_workspace_bytes(int N, int K, int P, int M) {
+    if (N < 1 || K < 1 || P < 1 || M < 1) return 0;
+    return rabit::gemm_workspace_bytes(N, K, P, M);
+}
+
+int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ldw, int P, const float *a,
+                      const float *b, uint32_t *packed, void *stream) {
+    if (w_dtype != RABIT_F32 && w_dtype != RABIT_BF16) return RABIT_ERR_INVALID_ARG;
+    if (!W || !a || !b || !packed) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || P < 1 || ldw < K) return RABIT_ERR_SHAPE;
+    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    int st = device_ctx(stream, ctx, nullptr);
+    if (st != RABIT_OK) return st;
+    return finish_launch(rabit::launch_derive_pack(ctx, W, w_dtype == RABIT_BF16, N, K, ldw, a, b, packed));
+}
+
+int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
+               const void *x, int x_dtype, int batch, int ldx, float *y, int ldy, void *stream) {
+    if (x_dtype != RABIT_F32 && x_dtype != RABIT_BF16) return RABIT_ERR_INVALID_ARG;
+    if (!packed || !a || !b || !x || !y) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || P < 1 || batch < 1 || batch > 16 || ldx < K || ldy < N)
+        return RABIT_ERR_SHAPE;
+    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16)) return RABIT_ERR_ALIGNMENT;
+    if (!aligned(x, x_dtype == RABIT_BF16 ? 2 : 4) || !aligned(y, 4)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    int st = device_ctx(stream, ctx, nullptr);
+    if (st != RABIT_OK) return st;
+    return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, x, x_dtype == RABIT_BF16,
+                                            batch, ldx, y, ldy));
+}
+
+int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
+               const uint16_t *x_bf16, int M, int ldx, float *y, int ldy, void *workspace,
+               size_t workspace_bytes, void *stream) {
+    if (!packed || !a || !b || !x_bf16 || !y) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || P < 1 || M < 1 || ldx < K || ldy < N) return RABIT_ERR_SHAPE;
+    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16) || !aligned(x_bf16, 16) || (ldx % 8) != 0 || !aligned(y, 4))
+        return RABIT_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < rabit::gemm_workspace_bytes(N, K, P, M))
+        return RABIT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
+    if (st != RABIT_OK) return st;
+    const uint64_t timeout_ns = wait_timeout_ns();
+    const int debug = env_flag("RABIT_TEST_SKIP_ONE_ARRIVE") ? 1 : 0;
+    return finish_launch(rabit::launch_gemm(ctx, packed, a, b, N, K, x_bf16, M, ldx, y, ldy,
+                                            workspace, fault, timeout_ns, debug));
+}
+
+int rabit_read_fault(void *stream, uint32_t *flags, int clear) {
+    rabit::LaunchCtx ctx;
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
+    if (st != RABIT_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(ctx.stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t v = 0;
+    e = cudaMemcpy(&v, fault, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (clear) {
+        e = cudaMemset(fault, 0, sizeof(uint32_t));
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (flags) *flags = v;
+    return v ? RABIT_ERR_TIMEOUT : RABIT_OK;
+}
+
+int rabit_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char *rabit_status_string(int status) {
+    switch (status) {
+        case RABIT_OK: return "RABIT_OK";
+        case RABIT_ERR_INVALID_ARG: return "RABIT_ERR_INVALID_ARG";
+        case RABIT_ERR_ALIGNMENT: return "RABIT_ERR_ALIGNMENT";
+        case RABIT_ERR_SHAPE: return "RABIT_ERR_SHAPE";
+        case RABIT_ERR_UNSUPPORTED: return "RABIT_ERR_UNSUPPORTED";
+        case RABIT_ERR_WORKSPACE: return "RABIT_ERR_WORKSPACE";
+        case RABIT_ERR_ARCH: return "RABIT_ERR_ARCH";
+        case RABIT_ERR_CUDA: return "RABIT_ERR_CUDA";
+        case RABIT_ERR_TIMEOUT: return "RABIT_ERR_TIMEOUT";
+        default: return "RABIT_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

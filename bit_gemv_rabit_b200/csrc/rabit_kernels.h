@@ -1,0 +1,34 @@
+// rabit_kernels.h -- host-side launchers shared between the librabit translation units.
+// Each launcher assumes its arguments were validated by the C ABI layer (rabit_abi.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace rabit {
+
+inline int64_t padded_cols(int K) { return ((static_cast<int64_t>(K) + 127) / 128) * 128; }
+
+// Launch configuration shared by every kernel launch: programmatic dependent launch lets a
+// kernel's prologue overlap the tail of the previous kernel on the same stream.
+struct LaunchCtx {
+    cudaStream_t stream;
+    int num_sms;
+    bool pdl;
+};
+
+cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16, int N, int K,
+                               int ldw, const float *a, const float *b, uint32_t *packed);
+
+cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
+                        const float *b, int N, int K, const void *x, bool x_bf16, int batch,
+                        int ldx, float *y, int ldy);
+
+size_t gemm_workspace_bytes(int N, int K, int P, int M);
+cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
+                        const float *b, int N, int K, const uint16_t *x, int M, int ldx,
+                        float *y, int ldy, void *workspace, uint32_t *fault_word,
+                        uint64_t timeout_ns, int debug_flags);
+
+}  // namespace rabit

@@ -1,0 +1,145 @@
+"""Python binding of librabit: argument marshalling only.
+
+Every function here has the name of a C entry point in include/rabit.h, takes torch CUDA
+tensors, passes their data pointers, sizes and torch's current CUDA stream to the C call,
+and raises :class:`RabitError` on a non-zero status.  No step of the layer runs here, and
+there is no fallback: if ``librabit.so`` is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librabit.so")
+
+RABIT_F32, RABIT_BF16 = 0, 1
+STATUS = {0: "RABIT_OK", -1: "RABIT_ERR_INVALID_ARG", -2: "RABIT_ERR_ALIGNMENT",
+          -3: "RABIT_ERR_SHAPE", -4: "RABIT_ERR_UNSUPPORTED", -5: "RABIT_ERR_WORKSPACE",
+          -6: "RABIT_ERR_ARCH", -7: "RABIT_ERR_CUDA", -8: "RABIT_ERR_TIMEOUT"}
+
+# (name, restype, argtypes) of every symbol include/rabit.h declares.
+_c, _p, _i, _sz = ctypes, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = [
+    ("rabit_packed_words", _sz, [_i, _i, _i]),
+    ("rabit_derive_pack", _i, [_p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
+    ("rabit_gemv", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _i, _p, _i, _p]),
+    ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
+    ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
+    ("rabit_read_fault", _i, [_p, ctypes.POINTER(ctypes.c_uint32), _i]),
+    ("rabit_last_cuda_error", _i, []),
+    ("rabit_status_string", ctypes.c_char_p, [_i]),
+]
+
+_lib = None
+
+
+class RabitError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        extra = ""
+        if status == -7 and _lib is not None:
+            extra = f" (cudaError {_lib.rabit_last_cuda_error()})"
+        super().__init__(f"{where}: {STATUS.get(status, status)}{extra}")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load librabit.so (raises OSError if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError(f"{path} not found: build it with `python -m bit_gemv_rabit_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, res, args in SIGNATURES:
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise RabitError(status, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RABIT_F32
+    if t.dtype == torch.bfloat16:
+        return RABIT_BF16
+    return 99  # rejected by the C layer as RABIT_ERR_INVALID_ARG
+
+
+def rabit_packed_words(N: int, K: int, P: int = 2) -> int:
+    return int(load().rabit_packed_words(N, K, P))
+
+
+def rabit_gemm_workspace_bytes(N: int, K: int, P: int, M: int) -> int:
+    return int(load().rabit_gemm_workspace_bytes(N, K, P, M))
+
+
+def rabit_derive_pack(W: torch.Tensor, a: torch.Tensor, b: torch.Tensor, packed: torch.Tensor,
+                      P: int = 2, stream=None) -> torch.Tensor:
+    """W [N][K] (row pitch W.stride(0)) fp32/bf16; a [P][N], b [P][K] fp32; packed uint32 out."""
+    N, K = W.shape
+    _check(load().rabit_derive_pack(_dptr(W), _dtype_code(W), N, K, W.stride(0), P, _dptr(a),
+                                    _dptr(b), _dptr(packed), _stream(stream)), "rabit_derive_pack")
+    return packed
+
+
+def rabit_gemv(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,
+               x: torch.Tensor, y: torch.Tensor, P: int = 2, stream=None) -> torch.Tensor:
+    """x [batch][K] bf16/fp32 (pitch x.stride(0)); y [batch][N] fp32 out (pitch y.stride(0))."""
+    batch = x.shape[0]
+    _check(load().rabit_gemv(_dptr(packed), _dptr(a), _dptr(b), N, K, P, _dptr(x), _dtype_code(x),
+                             batch, x.stride(0), _dptr(y), y.stride(0), _stream(stream)),
+           "rabit_gemv")
+    return y
+
+
+def rabit_gemm(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,
+               x: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor, P: int = 2,
+               stream=None) -> torch.Tensor:
+    """x [M][K] bf16 (pitch x.stride(0)); y [M][N] fp32 out; workspace: caller scratch."""
+    M = x.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().rabit_gemm(_dptr(packed), _dptr(a), _dptr(b), N, K, P, _dptr(x), M, x.stride(0),
+                             _dptr(y), y.stride(0), _dptr(workspace), ws_bytes, _stream(stream)),
+           "rabit_gemm")
+    return y
+
+
+def rabit_read_fault(clear: bool = True, stream=None) -> int:
+    """Synchronise and return the device fault word (0 = no bounded wait expired)."""
+    flags = ctypes.c_uint32(0)
+    st = load().rabit_read_fault(_stream(stream), ctypes.byref(flags), 1 if clear else 0)
+    if st not in (0, -8):
+        raise RabitError(st, "rabit_read_fault")
+    return int(flags.value)
+
+
+def rabit_status_string(status: int) -> str:
+    return load().rabit_status_string(status).decode()
+
+
+def alloc_packed(N: int, K: int, P: int = 2, device=None) -> torch.Tensor:
+    """A uint32 tensor of rabit_packed_words(N, K, P) words (torch allocates, 16 B aligned)."""
+    return torch.empty(rabit_packed_words(N, K, P), dtype=torch.uint32, device=device or "cuda")
+
+
+def alloc_gemm_workspace(N: int, K: int, P: int, M: int, device=None) -> torch.Tensor:
+    return torch.empty(rabit_gemm_workspace_bytes(N, K, P, M), dtype=torch.uint8,
+                       device=device or "cuda")

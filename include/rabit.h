@@ -1,0 +1,150 @@
+/*
+ * rabit.h -- C ABI of librabit, the RaBiT residual-binary linear layer on NVIDIA B200.
+ *
+ * The layer (RaBiT: Residual-Aware Binarization Training for Accurate and Efficient LLMs,
+ * arXiv 2602.05367, sec. 4.1 "Multi-bit Approximation via Stacking"):
+ *
+ *     y = sum_{k=1..P} a_k (.) ( S_k . ( b_k (.) x ) )
+ *
+ * S_k in {+1,-1}^{N x K} are sign planes, a_k (length N) a per-output scale and b_k
+ * (length K) a per-input scale (the paper's g_k and h_k).  The planes are derived in
+ * sequence from one shared full-precision weight W (sec. 4.2 "The Coupled Forward Pass"):
+ *     S_1 = sign(W),   R_1 = W - a_1 (.) S_1 (.) b_1,   S_2 = sign(R_1),
+ * with sign(v) = +1 unless v < 0 (so +0, -0, NaN and an exact residual tie give +1).
+ * Only the 2-path (2-bit) case, P = 2, is implemented.
+ *
+ * Conventions shared by every call:
+ *   - Every pointer argument is DEVICE memory owned by the caller (e.g. a torch tensor's
+ *     data_ptr()).  The library allocates no device memory and keeps no per-call state;
+ *     its only global state is a per-device fault word (rabit_read_fault) and cached
+ *     device attributes.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous:
+ *     they validate, enqueue and return.  Execution errors surface at the caller's next
+ *     synchronisation, as for any CUDA launch.
+ *   - Matrices are row-major; `ld*` arguments are row pitches in ELEMENTS.
+ *   - Every call returns a rabit_status (0 = success).  Arguments are validated before
+ *     anything is enqueued; a call that returns an error has enqueued nothing.  No call
+ *     aborts, throws or prints.  RABIT_ERR_CUDA leaves the cudaError_t in
+ *     rabit_last_cuda_error() (per calling thread).
+ *   - The device current on the calling thread must be an sm_100 (B200-class) GPU; any
+ *     other device gives RABIT_ERR_ARCH.
+ */
+#ifndef RABIT_H
+#define RABIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RABIT_API __attribute__((visibility("default")))
+#else
+#define RABIT_API
+#endif
+
+/* Element types accepted for W (derive) and x (gemv). */
+typedef enum rabit_dtype { RABIT_F32 = 0, RABIT_BF16 = 1 } rabit_dtype;
+
+typedef enum rabit_status {
+    RABIT_OK = 0,
+    RABIT_ERR_INVALID_ARG = -1,  /* null pointer, bad enum value */
+    RABIT_ERR_ALIGNMENT = -2,    /* a pointer or pitch breaks the stated alignment */
+    RABIT_ERR_SHAPE = -3,        /* N, K, M, batch or a pitch out of range */
+    RABIT_ERR_UNSUPPORTED = -4,  /* valid request this build does not implement (P != 2) */
+    RABIT_ERR_WORKSPACE = -5,    /* workspace missing or too small */
+    RABIT_ERR_ARCH = -6,         /* current device is not sm_100 */
+    RABIT_ERR_CUDA = -7,         /* a CUDA runtime call failed; see rabit_last_cuda_error() */
+    RABIT_ERR_TIMEOUT = -8       /* reported by rabit_read_fault: a bounded device wait expired */
+} rabit_status;
+
+/*
+ * Packed sign layout RABIT_LAYOUT_V2 (Appendix E.1 "Weight Packing": 32 columns per
+ * uint32 word, +1 -> bit 0, -1 -> bit 1, the 2-bit case's two words grouped as a uint2).
+ *   Kp = ceil(K/128)*128, Wr = Kp/32 groups of 32 columns per row;
+ *   column j sits at bit (j % 32) of group j/32, least significant bit first;
+ *   word(k, n, w) = (n*Wr + w)*2 + k    (path k in {0,1}, row n < N, group w < Wr).
+ * Rows are stored one after another (row pitch Kp/4 bytes), and inside a row the two
+ * paths' words of each 32-column group sit side by side.  Padding columns (j >= K) are 0;
+ * rows are not padded.  The buffer holds 2*N*Wr uint32 words and must be 16-byte aligned.
+ */
+#define RABIT_LAYOUT_V2 2
+RABIT_API size_t rabit_packed_words(int N, int K, int P);
+
+/*
+ * rabit_derive_pack -- sec. 4.2 "The Coupled Forward Pass", steps 1-3, followed by the
+ * Appendix E.1 packing.  For every n < N, j < K:
+ *     s1 = sign(W[n][j]);  r1 = W[n][j] - a[0][n]*s1*b[0][j];  s2 = sign(r1)
+ * r1 is formed with one rounding (fused multiply-add), so its sign is exact whenever the
+ * exact residual is nonzero and |a[0][n]*b[0][j]| >= 2^-100.  Writes every word of the
+ * packed buffer, padding columns included (so it never needs clearing).  Scales are read, never
+ * written: they stay caller-owned learnable parameters.
+ *   W       [N][ldw] fp32 (w_dtype RABIT_F32) or bf16 (RABIT_BF16), ldw >= K
+ *   a       [P][N] fp32, b [P][K] fp32 (only path 1 is read when P = 2)
+ *   packed  rabit_packed_words(N, K, P) uint32, 16-byte aligned (output)
+ * Errors: INVALID_ARG (null, bad dtype), SHAPE (N, K < 1, ldw < K), UNSUPPORTED (P != 2),
+ *         ALIGNMENT (packed), ARCH, CUDA.
+ */
+RABIT_API int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ldw, int P,
+                      const float *a, const float *b, uint32_t *packed, void *stream);
+
+/*
+ * rabit_gemv -- decode path, batch 1..16 (sec. 4.1 stacking executed per path as in
+ * Appendix E.1 "Compute Pipeline": paths computed in parallel, signs applied without
+ * multiplication, warp-level reduction):
+ *     y[beta][n] = sum_k a[k][n] * sum_j S_k[n][j] * b[k][j] * x[beta][j]
+ *   packed  RABIT_LAYOUT_V2 buffer of N x K, P paths (input)
+ *   a [P][N], b [P][K] fp32
+ *   x       [batch][ldx], bf16 (x_dtype RABIT_BF16) or fp32 (RABIT_F32), ldx >= K
+ *   y       [batch][ldy] fp32 (output, fully overwritten for n < N), ldy >= N
+ * Accuracy (normwise, max|y - y_exact| / max|y_exact|): <= 2e-3 for bf16 x, <= 1e-5 for
+ * fp32 x.  Errors: INVALID_ARG, SHAPE (batch outside 1..16, pitches), UNSUPPORTED,
+ * ALIGNMENT (packed), ARCH, CUDA.
+ */
+RABIT_API int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
+               const void *x, int x_dtype, int batch, int ldx, float *y, int ldy,
+               void *stream);
+
+/*
+ * rabit_gemm -- prefill / QAT forward path at large M (sec. 4.2: the forward pass uses
+ * W_hat^(2)), the same contraction as rabit_gemv for M tokens:
+ *     y[m][n] = sum_k a[k][n] * sum_j S_k[n][j] * b[k][j] * x[m][j]
+ * computed on the tensor cores: the signs are expanded to fp16 +-a[k][n] in tensor memory,
+ * the activations enter as fp16(x (.) b_k) and products accumulate in fp32.
+ *   packed  RABIT_LAYOUT_V2 buffer (input); a [P][N], b [P][K] fp32
+ *   x_bf16  [M][ldx] bf16, 16-byte aligned, ldx >= K and ldx % 8 == 0
+ *   y       [M][ldy] fp32 (output, fully overwritten for m < M, n < N), ldy >= N
+ *   workspace  scratch of at least rabit_gemm_workspace_bytes(N, K, P, M) bytes,
+ *              256-byte aligned, owned by the caller; contents need no initialisation
+ *              and are garbage afterwards.  Calls that share a workspace must not overlap.
+ * Accuracy: <= 2e-3 normwise, provided every |a[k][n]| lies in fp16's normal range
+ * [6.2e-5, 65504] and |x*b| < 65504.  Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT,
+ * WORKSPACE, ARCH, CUDA.  A device-side wait that expires (it cannot in correct operation)
+ * ends the kernel early and is reported by rabit_read_fault as RABIT_ERR_TIMEOUT.
+ */
+RABIT_API size_t rabit_gemm_workspace_bytes(int N, int K, int P, int M);
+RABIT_API int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
+               const uint16_t *x_bf16, int M, int ldx, float *y, int ldy,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * rabit_read_fault -- synchronise `stream` and read the current device's fault word
+ * (bit set by a kernel whose bounded wait expired).  Returns RABIT_OK when no fault is
+ * recorded, RABIT_ERR_TIMEOUT when one is, RABIT_ERR_CUDA on a CUDA failure.  `flags`
+ * (may be NULL) receives the raw word; clear != 0 resets it to 0 afterwards.
+ */
+RABIT_API int rabit_read_fault(void *stream, uint32_t *flags, int clear);
+
+/* Last cudaError_t seen by a librabit call on this thread (0 if none). */
+RABIT_API int rabit_last_cuda_error(void);
+
+/* Static, human-readable name of a rabit_status value. */
+RABIT_API const char *rabit_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RABIT_H */

@@ -45,13 +45,11 @@ def _load():
         i64, p = ctypes.c_int64, ctypes.c_void_p
         lib.oracle_derive_signs.argtypes = [p, i64, i64, i64, ctypes.c_int, p, p, i64, i64, p]
         lib.oracle_derive_signs.restype = None
-        lib.oracle_padded_rows.argtypes = [i64]
-        lib.oracle_padded_rows.restype = i64
         lib.oracle_padded_cols.argtypes = [i64]
         lib.oracle_padded_cols.restype = i64
         lib.oracle_packed_words.argtypes = [i64, i64, ctypes.c_int]
         lib.oracle_packed_words.restype = i64
-        lib.oracle_word_index.argtypes = [ctypes.c_int, i64, i64, i64, i64]
+        lib.oracle_word_index.argtypes = [ctypes.c_int, i64, i64, i64, ctypes.c_int]
         lib.oracle_word_index.restype = i64
         lib.oracle_pack.argtypes = [p, i64, i64, ctypes.c_int, p]
         lib.oracle_pack.restype = None
@@ -103,10 +101,6 @@ def derive_signs(W: np.ndarray, a: np.ndarray, b: np.ndarray, P: int = 2,
     return S
 
 
-def padded_rows(N: int) -> int:
-    return int(_load().oracle_padded_rows(N))
-
-
 def padded_cols(K: int) -> int:
     return int(_load().oracle_padded_cols(K))
 
@@ -115,13 +109,13 @@ def packed_words(N: int, K: int, P: int = 2) -> int:
     return int(_load().oracle_packed_words(N, K, P))
 
 
-def word_index(k: int, n: int, w: int, N: int, K: int) -> int:
-    """Position of (path k, row n, 32-column word w) in the RABIT_LAYOUT_V1 buffer."""
-    return int(_load().oracle_word_index(k, n, w, padded_rows(N), padded_cols(K)))
+def word_index(k: int, n: int, w: int, K: int, P: int = 2) -> int:
+    """Position of (path k, row n, 32-column word w) in the RABIT_LAYOUT_V2 buffer."""
+    return int(_load().oracle_word_index(k, n, w, K, P))
 
 
 def pack(S: np.ndarray) -> np.ndarray:
-    """Appendix E.1 packing of int8 signs [P][N][K] into RABIT_LAYOUT_V1 uint32 words."""
+    """Appendix E.1 packing of int8 signs [P][N][K] into RABIT_LAYOUT_V2 uint32 words."""
     S = np.ascontiguousarray(S, dtype=np.int8)
     P, N, K = S.shape
     out = np.empty(packed_words(N, K, P), dtype=np.uint32)

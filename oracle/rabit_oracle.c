@@ -14,15 +14,16 @@
  *   - sec. 4.2, "The Coupled Forward Pass", steps 1-3: B_1 = sign(W_FP),
  *     R_1 = W_FP - W_hat_1, B_2 = sign(R_1);
  *   - Appendix E.1, "Weight Packing": 32 columns per uint32, +1 -> bit 0, -1 -> bit 1,
- *     rows interleaved in warp-sized groups.
+ *     the paths' words of one 32-column group grouped together (uint2 for 2 bits).
  * In this library's names a_k is the per-output scale (g_k) and b_k the per-input scale (h_k).
  *
  * Readings where the pages are silent:
  *   - sign(v) = +1 unless v < 0, so +0, -0 and NaN binarize to +1 (the pages map only +-1);
  *   - column j of a 32-column group sits at bit (j % 32), least significant bit first;
- *   - the interleave is the RABIT_LAYOUT_V1 formula below (one 16-byte unit holds 128
- *     columns of one row; the 32 rows of a group are adjacent, so a 32-lane read of one
- *     unit per lane is 512 contiguous bytes).
+ *   - the arrangement is the RABIT_LAYOUT_V2 formula below: rows one after another, each
+ *     row's 32-column groups in order, each group holding the P paths' words side by side.
+ *     (The pages also interleave rows in warp-sized groups for a kernel that maps lanes to
+ *     rows; the kernel this oracle checks maps lanes to column groups, so rows stay whole.)
  *
  * Precision: every input is an fp32 (or bf16, widened exactly) value; the product a*b of
  * two fp32 values is exact in binary64, so the residual W - a*s*b is rounded once and its
@@ -68,48 +69,50 @@ ORACLE_API void oracle_derive_signs(const double *W, int64_t N, int64_t K, int64
     }
 }
 
-/* Padded sizes of the packed layout: rows to a multiple of 32, columns to a multiple of 128. */
-ORACLE_API int64_t oracle_padded_rows(int64_t N) { return ((N + 31) / 32) * 32; }
+/* Padded column count of the packed layout: columns to a multiple of 128.  Rows are not padded. */
 ORACLE_API int64_t oracle_padded_cols(int64_t K) { return ((K + 127) / 128) * 128; }
+
+/* Words of one 32-column group: the P paths' words side by side, padded to a power of two
+   (P = 2 -> 2 words, the "uint2" grouping of Appendix E.1). */
+static int64_t oracle_group_words(int P) { return P <= 1 ? 1 : (P == 2 ? 2 : 4); }
+
 ORACLE_API int64_t oracle_packed_words(int64_t N, int64_t K, int P)
 {
-    return (int64_t)P * oracle_padded_rows(N) * (oracle_padded_cols(K) / 32);
+    return N * (oracle_padded_cols(K) / 32) * oracle_group_words(P);
 }
 
 /*
- * RABIT_LAYOUT_V1 word index of (path k, row n, 32-column word w):
- *   unit  = (k * Np/32 + n/32) * Kp/128 + w/4      (16-byte unit = 4 words = 128 columns)
- *   index = unit * 128 + (n % 32) * 4 + (w % 4)      (32 rows of a group are adjacent)
+ * RABIT_LAYOUT_V2 word index of (path k, row n, 32-column word w), P paths:
+ *   index = (n * (Kp/32) + w) * G + k,   G = words per group (2 for P = 2)
+ * i.e. rows are stored one after another; inside a row, each 32-column group holds the
+ * P paths' words next to each other (Appendix E.1 groups the 2-bit case's words as uint2).
  */
-ORACLE_API int64_t oracle_word_index(int k, int64_t n, int64_t w, int64_t Np, int64_t Kp)
+ORACLE_API int64_t oracle_word_index(int k, int64_t n, int64_t w, int64_t K, int P)
 {
-    int64_t unit = ((int64_t)k * (Np / 32) + n / 32) * (Kp / 128) + w / 4;
-    return unit * 128 + (n % 32) * 4 + (w % 4);
+    return (n * (oracle_padded_cols(K) / 32) + w) * oracle_group_words(P) + k;
 }
 
 /*
  * Pack signs (Appendix E.1 "Weight Packing"): bit (j % 32) of word j/32 is 1 iff S = -1.
- * Padding rows and padding columns stay 0.  S is [P][N][K]; out has oracle_packed_words().
+ * Padding columns (and the padding word of a 3-path group) stay 0.  S is [P][N][K]; out has oracle_packed_words().
  */
 ORACLE_API void oracle_pack(const int8_t *S, int64_t N, int64_t K, int P, uint32_t *out)
 {
-    const int64_t Np = oracle_padded_rows(N), Kp = oracle_padded_cols(K);
     memset(out, 0, sizeof(uint32_t) * (size_t)oracle_packed_words(N, K, P));
     for (int k = 0; k < P; ++k)
         for (int64_t n = 0; n < N; ++n)
             for (int64_t j = 0; j < K; ++j)
                 if (S[((int64_t)k * N + n) * K + j] == -1)
-                    out[oracle_word_index(k, n, j / 32, Np, Kp)] |= (uint32_t)1u << (j % 32);
+                    out[oracle_word_index(k, n, j / 32, K, P)] |= (uint32_t)1u << (j % 32);
 }
 
 /* Inverse of oracle_pack: bit 1 -> -1, bit 0 -> +1.  S is [P][N][K]. */
 ORACLE_API void oracle_unpack(const uint32_t *packed, int64_t N, int64_t K, int P, int8_t *S)
 {
-    const int64_t Np = oracle_padded_rows(N), Kp = oracle_padded_cols(K);
     for (int k = 0; k < P; ++k)
         for (int64_t n = 0; n < N; ++n)
             for (int64_t j = 0; j < K; ++j) {
-                uint32_t word = packed[oracle_word_index(k, n, j / 32, Np, Kp)];
+                uint32_t word = packed[oracle_word_index(k, n, j / 32, K, P)];
                 S[((int64_t)k * N + n) * K + j] = ((word >> (j % 32)) & 1u) ? (int8_t)-1 : (int8_t)1;
             }
 }

@@ -1,0 +1,113 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments before touching the GPU.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import oracle
+from bit_gemv_rabit_b200 import build as rbuild
+from bit_gemv_rabit_b200 import rabit
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+OK, INVALID, ALIGN, SHAPE, UNSUP, WS, ARCH, CUDA = 0, -1, -2, -3, -4, -5, -6, -7
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+P = ctypes.c_void_p
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rbuild.build()
+    return rabit.load()
+
+
+def declared_symbols():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        names |= set(re.findall(r"RABIT_API\s+[\w\s\*]+?\b(rabit_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert {"rabit_derive_pack", "rabit_gemv", "rabit_gemm"} <= names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert names == {s[0] for s in rabit.SIGNATURES}
+
+
+def test_packed_words_matches_layout_definition(lib):
+    for N, K in [(1, 1), (32, 128), (33, 129), (4096, 4096), (11008, 4096), (4096, 14336)]:
+        assert lib.rabit_packed_words(N, K, 2) == oracle.packed_words(N, K, 2)
+    assert lib.rabit_packed_words(0, 5, 2) == 0
+    assert lib.rabit_gemm_workspace_bytes(4096, 4096, 2, 2048) == 2 * 2048 * 4096 * 2
+    assert lib.rabit_gemm_workspace_bytes(10, 200, 2, 3) == 2 * 3 * 256 * 2
+
+
+def test_status_strings(lib):
+    assert rabit.rabit_status_string(0) == "RABIT_OK"
+    assert rabit.rabit_status_string(-8) == "RABIT_ERR_TIMEOUT"
+    assert rabit.rabit_status_string(123) == "RABIT_ERR_UNKNOWN"
+
+
+def test_derive_pack_validation(lib):
+    f = lib.rabit_derive_pack
+    assert f(P(FAKE), 7, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None) == INVALID   # dtype
+    assert f(None, 0, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None) == INVALID      # null W
+    assert f(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), None, None) == INVALID      # null out
+    assert f(P(FAKE), 0, 0, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None) == SHAPE     # N = 0
+    assert f(P(FAKE), 0, 4, 4, 3, 2, P(FAKE), P(FAKE), P(FAKE), None) == SHAPE     # ldw < K
+    assert f(P(FAKE), 0, 4, 4, 4, 3, P(FAKE), P(FAKE), P(FAKE), None) == UNSUP     # P = 3
+    assert f(P(FAKE), 0, 4, 4, 4, 1, P(FAKE), P(FAKE), P(FAKE), None) == UNSUP     # P = 1
+    assert f(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE + 4), None) == ALIGN
+
+
+def test_gemv_validation(lib):
+    f = lib.rabit_gemv
+    args = lambda **kw: [P(kw.get("packed", FAKE)), P(FAKE), P(FAKE), kw.get("N", 8), kw.get("K", 8),
+                         kw.get("P", 2), P(kw.get("x", FAKE)), kw.get("xd", 1), kw.get("batch", 1),
+                         kw.get("ldx", 8), P(kw.get("y", FAKE)), kw.get("ldy", 8), None]
+    assert f(*args(xd=5)) == INVALID
+    assert f(*args(packed=0)) == INVALID
+    assert f(*args(y=0)) == INVALID
+    assert f(*args(batch=0)) == SHAPE
+    assert f(*args(batch=17)) == SHAPE
+    assert f(*args(ldx=7)) == SHAPE
+    assert f(*args(ldy=7)) == SHAPE
+    assert f(*args(K=0)) == SHAPE
+    assert f(*args(P=3)) == UNSUP
+    assert f(*args(packed=FAKE + 8)) == ALIGN
+    assert f(*args(x=FAKE + 1)) == ALIGN
+    assert f(*args(y=FAKE + 2)) == ALIGN
+
+
+def test_gemm_validation(lib):
+    f = lib.rabit_gemm
+    need = lib.rabit_gemm_workspace_bytes(8, 16, 2, 4)
+    args = lambda **kw: [P(kw.get("packed", FAKE)), P(FAKE), P(FAKE), kw.get("N", 8), kw.get("K", 16),
+                         kw.get("P", 2), P(kw.get("x", FAKE)), kw.get("M", 4), kw.get("ldx", 16),
+                         P(FAKE), kw.get("ldy", 8), P(kw.get("ws", FAKE)), kw.get("wsb", need), None]
+    assert f(*args(x=0)) == INVALID
+    assert f(*args(M=0)) == SHAPE
+    assert f(*args(ldx=8)) == SHAPE
+    assert f(*args(ldy=4)) == SHAPE
+    assert f(*args(P=1)) == UNSUP
+    assert f(*args(x=FAKE + 8)) == ALIGN            # x must be 16-byte aligned
+    assert f(*args(ldx=20)) == ALIGN                # pitch must keep rows 16-byte aligned
+    assert f(*args(ws=0)) == WS
+    assert f(*args(wsb=need - 1)) == WS
+    assert f(*args(ws=FAKE + 16)) == ALIGN          # workspace 256-byte alignment
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="valid arguments would launch on a GPU")
+def test_valid_arguments_without_gpu_fail_cleanly(lib):
+    st = lib.rabit_derive_pack(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None)
+    assert st in (CUDA, ARCH)
+    flags = ctypes.c_uint32(0)
+    assert lib.rabit_read_fault(None, ctypes.byref(flags), 0) in (CUDA, ARCH)

@@ -1,0 +1,101 @@
+"""GPU parity at the full workload sizes, in the launch configurations the benchmark times.
+
+The whole matrix goes through the CUDA path; the oracle checks a seeded sample of rows
+(first, last and random ones) one by one: their packed words bit-exactly, their outputs
+within the normwise tolerance.  Workloads: the Llama-2-7B decode layer set (batch 1), the
+Llama-3-8B decode set with outliers (batch 1/4/8/16), the Llama-3-8B MLP prefill GEMM at
+M=2048 and the Llama-3-70B MLP QAT step (derive + GEMM at M=4096).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_gemv_rabit_b200 import inputs
+from bit_gemv_rabit_b200 import rabit
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+TOL = 2e-3
+
+
+def normwise(y, ref):
+    return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-300))
+
+
+def sample_rows(N, seed, count=48):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(N, size=min(count, N), replace=False).tolist()) | {0, N - 1}
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from bit_gemv_rabit_b200 import build
+    build.build()
+    rabit.load()
+    rabit.rabit_read_fault(clear=True)
+    yield
+    assert rabit.rabit_read_fault(clear=True) == 0
+
+
+def derive_and_check(W, a, b, rows):
+    """GPU derive of the whole W; bit-exact check of the sampled rows; returns (packed, S_rows)."""
+    N, K = W.shape
+    packed = rabit.alloc_packed(N, K)
+    rabit.rabit_derive_pack(torch.from_numpy(W).cuda(), torch.from_numpy(a).cuda(),
+                            torch.from_numpy(b).cuda(), packed)
+    torch.cuda.synchronize()
+    per_row = oracle.packed_words(1, K)
+    host = packed.cpu().numpy().reshape(N, per_row)
+    S_rows = np.concatenate([oracle.derive_signs(W, a, b, rows=(int(r), int(r) + 1)) for r in rows], axis=1)
+    np.testing.assert_array_equal(host[rows], oracle.pack(S_rows).reshape(len(rows), per_row))
+    return packed, S_rows
+
+
+def decode_set(workload):
+    spec = inputs.WORKLOADS[workload]
+    for idx, (name, N, K) in enumerate(spec["set"]):
+        seed = inputs.seed_for(spec["cfg"], idx)
+        W = inputs.weight(seed, N, K, sigma=spec["sigma"], outlier_frac=spec["w_outliers"])
+        a, b = inputs.scales(seed, W)
+        yield name, N, K, seed, W, a, b, spec
+
+
+@pytest.mark.parametrize("workload", ["single_4096x4096_b1", "llama2_7b_decode_b1", "llama3_8b_decode"])
+def test_decode_sets_full_size(workload):
+    for name, N, K, seed, W, a, b, spec in decode_set(workload):
+        rows = sample_rows(N, seed)
+        packed, S_rows = derive_and_check(W, a, b, rows)
+        at, bt = torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()
+        for B in spec["batches"]:
+            x = inputs.activations(seed, B, K, channel_outlier_frac=spec["x_outliers"])
+            y = torch.empty((B, N), device="cuda")
+            rabit.rabit_gemv(packed, at, bt, N, K, bf16_dev(x), y)
+            torch.cuda.synchronize()
+            ref = oracle.layer(S_rows, a, b, x, rows=rows, N=N)
+            err = normwise(y.cpu().numpy()[:, rows].astype(np.float64), ref)
+            assert err <= TOL, (name, B, err)
+
+
+@pytest.mark.parametrize("workload", ["llama3_8b_mlp_prefill_m2048", "llama3_70b_mlp_qat_m4096"])
+def test_gemm_workloads_full_size(workload):
+    for name, N, K, seed, W, a, b, spec in decode_set(workload):
+        rows = sample_rows(N, seed, count=16)
+        packed, S_rows = derive_and_check(W, a, b, rows)
+        M = spec["batches"][0]
+        x = inputs.activations(seed, M, K, channel_outlier_frac=spec["x_outliers"])
+        y = torch.empty((M, N), device="cuda")
+        ws = rabit.alloc_gemm_workspace(N, K, 2, M)
+        rabit.rabit_gemm(packed, torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), N, K,
+                         bf16_dev(x), y, ws)
+        torch.cuda.synchronize()
+        ref = oracle.layer(S_rows, a, b, x, rows=rows, N=N)
+        err = normwise(y.cpu().numpy()[:, rows].astype(np.float64), ref)
+        assert err <= TOL, (name, err)

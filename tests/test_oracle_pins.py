@@ -203,9 +203,9 @@ def test_pack_hand_built_words():
     S[0, 5, :32] = np.where(np.arange(32) % 2 == 1, -1, 1)  # alternating: bits 1,3,5,... set
     packed = oracle.pack(S)
     assert packed.size == P * N * K // 32
-    assert packed[oracle.word_index(0, 0, 0, N, K)] == 0x00000000
-    assert packed[oracle.word_index(1, 7, 3, N, K)] == 0xFFFFFFFF
-    assert packed[oracle.word_index(0, 5, 0, N, K)] == 0xAAAAAAAA
+    assert packed[oracle.word_index(0, 0, 0, K)] == 0x00000000
+    assert packed[oracle.word_index(1, 7, 3, K)] == 0xFFFFFFFF
+    assert packed[oracle.word_index(0, 5, 0, K)] == 0xAAAAAAAA
     # column 0 is the least significant bit
     S2 = np.ones((1, 1, 1), dtype=np.int8)
     S2[0, 0, 0] = -1
@@ -214,17 +214,20 @@ def test_pack_hand_built_words():
 
 
 def test_layout_formula_hand_offsets():
-    # N=40 -> Np=64 (2 row groups); K=200 -> Kp=256 (2 units of 128 columns per row).
+    # N=40, K=200 -> Kp=256: 8 groups of 32 columns per row, 2 words (paths) per group.
     N, K = 40, 200
-    assert oracle.padded_rows(N) == 64 and oracle.padded_cols(K) == 256
-    assert oracle.packed_words(N, K, 2) == 2 * 64 * 256 // 32
-    # (k, n, w) -> ((k*2 + n//32)*2 + w//4)*128 + (n%32)*4 + w%4, evaluated by hand:
-    assert oracle.word_index(0, 0, 0, N, K) == 0
-    assert oracle.word_index(0, 1, 0, N, K) == 4
-    assert oracle.word_index(0, 0, 3, N, K) == 3
-    assert oracle.word_index(0, 0, 4, N, K) == 128
-    assert oracle.word_index(0, 33, 5, N, K) == 384 + 4 + 1
-    assert oracle.word_index(1, 39, 7, N, K) == 896 + 28 + 3
+    assert oracle.padded_cols(K) == 256
+    assert oracle.packed_words(N, K, 2) == 40 * 8 * 2
+    # (k, n, w) -> (n*8 + w)*2 + k, evaluated by hand:
+    assert oracle.word_index(0, 0, 0, K) == 0
+    assert oracle.word_index(1, 0, 0, K) == 1
+    assert oracle.word_index(0, 0, 3, K) == 6
+    assert oracle.word_index(0, 1, 0, K) == 16
+    assert oracle.word_index(0, 33, 5, K) == 538
+    assert oracle.word_index(1, 39, 7, K) == 639      # the last word of the buffer
+    # three paths: groups of 4 words (one padding word), (n*8 + w)*4 + k
+    assert oracle.packed_words(N, K, 3) == 40 * 8 * 4
+    assert oracle.word_index(2, 1, 2, K, P=3) == 42
 
 
 def test_pack_unpack_roundtrip_and_padding_zero():
