@@ -33,6 +33,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "rabit.h"
 #include "rabit_device.cuh"
 #include "rabit_kernels.h"
 
@@ -326,6 +327,30 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 }  // namespace
+
+// Scratch for rabit_gemm_noalloc: a fixed buffer in the library's device image, so callers
+// that may not allocate device memory can still run the GEMM.  In host code this name is
+// only a host-side stand-in, never a device address: gemm_noalloc_scratch() looks up the
+// device address, and that address is what the kernels receive.
+static __device__ __align__(256) uint8_t g_gemm_noalloc_scratch[RABIT_GEMM_NOALLOC_SCRATCH_BYTES];
+
+cudaError_t gemm_noalloc_scratch(void **ptr, size_t *bytes) {
+    // Looked up once per device, with that device current (the first call on each device).
+    static void *cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!cache[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        cache[dev] = p;
+    }
+    *ptr = cache[dev];
+    *bytes = sizeof(g_gemm_noalloc_scratch);
+    return cudaSuccess;
+}
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M) {
     (void)N;

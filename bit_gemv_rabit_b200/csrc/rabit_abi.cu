@@ -150,6 +150,32 @@ int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, in
                                             workspace, fault, timeout_ns, debug));
 }
 
+// For callers that may not allocate device memory: the scratch comes from the library's
+// fixed buffer instead of a caller workspace (see include/rabit.h).
+int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
+                       const uint16_t *x_bf16, int M, int ldx, float *y, int ldy, void *stream) {
+    if (!packed || !a || !b || !x_bf16 || !y) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || P < 1 || M < 1 || ldx < K || ldy < N) return RABIT_ERR_SHAPE;
+    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16) || !aligned(x_bf16, 16) || (ldx % 8) != 0 || !aligned(y, 4))
+        return RABIT_ERR_ALIGNMENT;
+    const size_t need = rabit::gemm_workspace_bytes(N, K, P, M);
+    if (need > RABIT_GEMM_NOALLOC_SCRATCH_BYTES) return RABIT_ERR_WORKSPACE;
+    rabit::LaunchCtx ctx;
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
+    if (st != RABIT_OK) return st;
+    void *scratch = nullptr;
+    size_t scratch_bytes = 0;
+    cudaError_t e = rabit::gemm_noalloc_scratch(&scratch, &scratch_bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (need > scratch_bytes) return RABIT_ERR_WORKSPACE;
+    const uint64_t timeout_ns = wait_timeout_ns();
+    const int debug = env_flag("RABIT_TEST_SKIP_ONE_ARRIVE") ? 1 : 0;
+    return finish_launch(rabit::launch_gemm(ctx, packed, a, b, N, K, x_bf16, M, ldx, y, ldy,
+                                            scratch, fault, timeout_ns, debug));
+}
+
 int rabit_read_fault(void *stream, uint32_t *flags, int clear) {
     rabit::LaunchCtx ctx;
     uint32_t *fault = nullptr;

@@ -26,6 +26,8 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
                         int ldx, float *y, int ldy);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
+// Device address and size of the library's fixed GEMM scratch buffer (rabit_gemm_noalloc).
+cudaError_t gemm_noalloc_scratch(void **ptr, size_t *bytes);
 cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
                         const float *b, int N, int K, const uint16_t *x, int M, int ldx,
                         float *y, int ldy, void *workspace, uint32_t *fault_word,

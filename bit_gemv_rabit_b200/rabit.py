@@ -28,6 +28,7 @@ SIGNATURES = [
     ("rabit_gemv", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _i, _p, _i, _p]),
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
+    ("rabit_gemm_noalloc", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p]),
     ("rabit_read_fault", _i, [_p, ctypes.POINTER(ctypes.c_uint32), _i]),
     ("rabit_last_cuda_error", _i, []),
     ("rabit_status_string", ctypes.c_char_p, [_i]),
@@ -119,6 +120,18 @@ def rabit_gemm(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K
     _check(load().rabit_gemm(_dptr(packed), _dptr(a), _dptr(b), N, K, P, _dptr(x), M, x.stride(0),
                              _dptr(y), y.stride(0), _dptr(workspace), ws_bytes, _stream(stream)),
            "rabit_gemm")
+    return y
+
+
+def rabit_gemm_noalloc(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,
+                       x: torch.Tensor, y: torch.Tensor, P: int = 2, stream=None) -> torch.Tensor:
+    """rabit_gemm without a workspace, for callers that may not allocate device memory: the
+    scratch is the library's fixed buffer (RABIT_GEMM_NOALLOC_SCRATCH_BYTES per device).
+    Calls that may overlap on the GPU race on that buffer; order them on one stream."""
+    M = x.shape[0]
+    _check(load().rabit_gemm_noalloc(_dptr(packed), _dptr(a), _dptr(b), N, K, P, _dptr(x), M,
+                                     x.stride(0), _dptr(y), y.stride(0), _stream(stream)),
+           "rabit_gemm_noalloc")
     return y
 
 

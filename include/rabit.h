@@ -130,6 +130,34 @@ RABIT_API int rabit_gemm(const uint32_t *packed, const float *a, const float *b,
                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * rabit_gemm_noalloc -- the same computation as rabit_gemm, for callers that are not allowed
+ * to allocate device memory and so cannot hand rabit_gemm a workspace.  Examples: a plugin
+ * loaded into an inference engine that owns every device allocation and gives the plugin
+ * no allocator, or a latency-critical serving loop that must never call cudaMalloc (it can
+ * synchronise the whole device and fails while another thread captures a stream in global
+ * mode).  The paper has no counterpart to this call; it exists only for such callers.
+ *
+ * The scratch rabit_gemm would take from `workspace` (the fp16 x (.) b_k operand) lives
+ * instead in one fixed device buffer of RABIT_GEMM_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads librabit holds until the process exits.  Nothing is
+ * allocated by this call.
+ *   - Requests that need more scratch than that (rabit_gemm_workspace_bytes(N, K, P, M) >
+ *     RABIT_GEMM_NOALLOC_SCRATCH_BYTES, e.g. more than 512 tokens at K = 4096) are rejected
+ *     with RABIT_ERR_WORKSPACE before anything is enqueued; use rabit_gemm for them.
+ *   - All calls on a device share the one buffer and leave their data in it.  The call
+ *     overwrites every byte it reads, so nothing needs clearing, but two calls that can run
+ *     at the same time on the GPU (different streams without ordering between them) race on
+ *     the buffer and give wrong results: order such calls on one stream or with events.
+ *   - The first call on each device looks up the buffer's device address; make that first
+ *     call before any stream capture begins.
+ * Arguments, accuracy and the other errors are those of rabit_gemm.
+ */
+#define RABIT_GEMM_NOALLOC_SCRATCH_BYTES (8u << 20)
+RABIT_API int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, int N,
+                                 int K, int P, const uint16_t *x_bf16, int M, int ldx, float *y,
+                                 int ldy, void *stream);
+
+/*
  * rabit_read_fault -- synchronise `stream` and read the current device's fault word
  * (bit set by a kernel whose bounded wait expired).  Returns RABIT_OK when no fault is
  * recorded, RABIT_ERR_TIMEOUT when one is, RABIT_ERR_CUDA on a CUDA failure.  `flags`
