@@ -73,7 +73,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if force or jobs or _stale(LIB, objs):
         tmp = LIB + f".tmp{os.getpid()}"
         cmd = [NVCC, *ARCH_FLAGS, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC",
-               *objs, "-o", tmp]
+               "-Xlinker", "-z", "-Xlinker", "defs", *objs, "-o", tmp]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)

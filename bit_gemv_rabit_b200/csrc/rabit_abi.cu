@@ -123,10 +123,11 @@ int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, in
     if (!aligned(packed, 16)) return RABIT_ERR_ALIGNMENT;
     if (!aligned(x, x_dtype == RABIT_BF16 ? 2 : 4) || !aligned(y, 4)) return RABIT_ERR_ALIGNMENT;
     rabit::LaunchCtx ctx;
-    int st = device_ctx(stream, ctx, nullptr);
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
     return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, x, x_dtype == RABIT_BF16,
-                                            batch, ldx, y, ldy));
+                                            batch, ldx, y, ldy, fault, wait_timeout_ns()));
 }
 
 int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,

@@ -21,6 +21,7 @@ enum : uint32_t {
     FAULT_GEMM_WAIT_EXPAND = 1u << 2,
     FAULT_GEMM_WAIT_EPILOGUE = 1u << 3,
     FAULT_GEMM_DRAIN = 1u << 4,
+    FAULT_GEMV_WAIT_COPY = 1u << 5,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

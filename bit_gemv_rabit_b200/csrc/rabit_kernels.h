@@ -23,7 +23,7 @@ cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16,
 
 cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
                         const float *b, int N, int K, const void *x, bool x_bf16, int batch,
-                        int ldx, float *y, int ldy);
+                        int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
 // Device address and size of the library's fixed GEMM scratch buffer (rabit_gemm_noalloc).
