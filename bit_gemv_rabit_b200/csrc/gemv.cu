@@ -54,6 +54,8 @@ struct GemvArgs {
     int nchunks;           // 32-group chunks of a row
     int wpr;               // warps across a row (each takes chunks wpr apart)
     int streams;           // warps along rows
+    int vec_x;             // x rows 16-byte aligned: 16-byte loads of 8 columns
+    int vec_b;             // both b rows 16-byte aligned
 };
 
 struct SmemLayout {
@@ -106,6 +108,57 @@ __device__ __forceinline__ float load_x(const void *x, int64_t idx) {
     } else {
         const unsigned short bits = __ldg(reinterpret_cast<const unsigned short *>(x) + idx);
         return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+    }
+}
+
+// Loads of one z task: 8 columns j0..j0+7 of x (batch row beta) and of both b rows.
+// Columns at or past K read as 0 (the padding of the last group).
+template <bool kF32X>
+__device__ __forceinline__ void load_ztask(const GemvArgs &p, int beta, int j0, bool on,
+                                           float (&xv)[8], float (&bv)[2][8]) {
+    const int64_t xrow = static_cast<int64_t>(beta) * p.ldx;
+    if (on && j0 + 8 <= p.K) {
+        if (p.vec_x) {
+            if constexpr (kF32X) {
+                const float4 *src = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.x) + xrow + j0);
+                const float4 u0 = __ldg(src), u1 = __ldg(src + 1);
+                xv[0] = u0.x; xv[1] = u0.y; xv[2] = u0.z; xv[3] = u0.w;
+                xv[4] = u1.x; xv[5] = u1.y; xv[6] = u1.z; xv[7] = u1.w;
+            } else {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                    reinterpret_cast<const unsigned short *>(p.x) + xrow + j0));
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    xv[2 * i] = __uint_as_float(w4[i] << 16);
+                    xv[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) xv[i] = load_x<kF32X>(p.x, xrow + j0 + i);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const float *brow = p.b + static_cast<int64_t>(k) * p.K + j0;
+            if (p.vec_b) {
+                const float4 u0 = __ldg(reinterpret_cast<const float4 *>(brow));
+                const float4 u1 = __ldg(reinterpret_cast<const float4 *>(brow) + 1);
+                bv[k][0] = u0.x; bv[k][1] = u0.y; bv[k][2] = u0.z; bv[k][3] = u0.w;
+                bv[k][4] = u1.x; bv[k][5] = u1.y; bv[k][6] = u1.z; bv[k][7] = u1.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bv[k][i] = __ldg(brow + i);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool ok = on && j0 + i < p.K;
+            xv[i] = ok ? load_x<kF32X>(p.x, xrow + j0 + i) : 0.0f;
+            bv[0][i] = ok ? __ldg(p.b + j0 + i) : 0.0f;
+            bv[1][i] = ok ? __ldg(p.b + p.K + j0 + i) : 0.0f;
+        }
     }
 }
 
@@ -203,80 +256,91 @@ gemv_kernel(const GemvArgs p) {
         for (int beta = 0; beta < p.batch; ++beta) {
             // ---- z_k = x (.) b_k over the whole row, quantised per 32-column group and path.
             // 4 consecutive threads per group, 8 columns each; x is read once for both paths.
+            // The loads of kZBatch tasks are issued before any of them is used, and a's values
+            // for the pass are fetched alongside, so the stage waits on memory about once.
+            float2 apre = make_float2(0.0f, 0.0f);
+            if (beta == 0 && tid < prows) apre = make_float2(__ldg(p.a + pr0 + tid), __ldg(p.a + p.N + pr0 + tid));
+            constexpr int kZBatch = 2;
             const int ztasks = 4 * p.Wr;
-            for (int t = tid; t < ((ztasks + 31) & ~31); t += nthreads) {
-                const bool on = t < ztasks;
-                const int q = t & 3;
-                const int gloc = on ? (t >> 2) : 0;
-                float xv[8], z[2][8];
+            const int ztasks_pad = (ztasks + 31) & ~31;
+            for (int t0 = tid; t0 < ztasks_pad; t0 += kZBatch * nthreads) {
+                float xv[kZBatch][8], zv[kZBatch][2][8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int j = gloc * 32 + 8 * q + i;
-                    const bool ok = on && j < p.K;
-                    xv[i] = ok ? load_x<kF32X>(p.x, static_cast<int64_t>(beta) * p.ldx + j) : 0.0f;
-                    z[0][i] = ok ? __ldg(p.b + j) : 0.0f;
-                    z[1][i] = ok ? __ldg(p.b + p.K + j) : 0.0f;
+                for (int u = 0; u < kZBatch; ++u) {
+                    const int t = t0 + u * nthreads;
+                    load_ztask<kF32X>(p, beta, (t >> 2) * 32 + 8 * (t & 3), t < ztasks, xv[u], zv[u]);
                 }
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    float m = 0.0f;
+                for (int u = 0; u < kZBatch; ++u) {
+                    const int t = t0 + u * nthreads;
+                    if (t - tid >= ztasks_pad) break;   // warp-uniform: t - tid is the same for all lanes
+                    const bool on = t < ztasks;
+                    const int q = t & 3;
+                    const int gloc = on ? (t >> 2) : 0;
+                    const int h = q >> 1, half = q & 1;  // columns 8q..8q+7 of the group
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        z[k][i] *= xv[i];
-                        m = fmaxf(m, fabsf(z[k][i]));
-                    }
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                    // power-of-two scale 2^e with m * 2^e <= kMaxQ (15-bit, or 29-bit for fp32 x)
-                    constexpr int kTop = kF32X ? 27 : 13;
-                    const float kMaxQ = kF32X ? 268435455.0f : 16383.0f;
-                    const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xFFu) - 127;
-                    int e = min(127, max(-126, kTop - E));
-                    float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-                    if (m * sc > kMaxQ) { --e; sc *= 0.5f; }
-                    int zsum[kSlices];
+                    for (int k = 0; k < 2; ++k) {
+                        float m = 0.0f;
 #pragma unroll
-                    for (int s = 0; s < kSlices; ++s) zsum[s] = 0;
-                    const int h = q >> 1, half = q & 1;       // columns 8q..8q+7 of the group
+                        for (int i = 0; i < 8; ++i) {
+                            zv[u][k][i] *= xv[u][i];
+                            m = fmaxf(m, fabsf(zv[u][k][i]));
+                        }
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                        // power-of-two scale 2^e with m * 2^e <= kMaxQ (15-bit, or 29-bit for fp32 x)
+                        constexpr int kTop = kF32X ? 27 : 13;
+                        const float kMaxQ = kF32X ? 268435455.0f : 16383.0f;
+                        const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xFFu) - 127;
+                        int e = min(127, max(-126, kTop - E));
+                        float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+                        if (m * sc > kMaxQ) { --e; sc *= 0.5f; }
+                        int zsum[kSlices];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int sh = i >> 1, jj = i & 1;
-                        const int pair = sh * 4 + jj * 2 + h;
-                        const int zq = __float2int_rn(z[k][i] * sc);
-                        int part[kSlices];
-                        if constexpr (kF32X) {
-                            part[0] = (zq + (1 << 13)) >> 14;       // high 15-bit slice
-                            part[1] = zq - (part[0] << 14);         // low slice, in [-2^13, 2^13)
-                        } else {
-                            part[0] = zq;
+                        for (int s = 0; s < kSlices; ++s) zsum[s] = 0;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int sh = i >> 1, jj = i & 1;
+                            const int pair = sh * 4 + jj * 2 + h;
+                            int part[kSlices];
+                            if constexpr (kF32X) {
+                                const int zq = __float2int_rn(zv[u][k][i] * sc);
+                                part[0] = (zq + (1 << 13)) >> 14;       // high 15-bit slice
+                                part[1] = zq - (part[0] << 14);         // low slice, in [-2^13, 2^13)
+                            } else {
+                                // round to nearest even by adding 1.5 * 2^23 (|z * 2^e| < 2^22)
+                                part[0] = __float_as_int(fmaf(zv[u][k][i], sc, 12582912.0f)) - 0x4B400000;
+                            }
+#pragma unroll
+                            for (int s = 0; s < kSlices; ++s) {
+                                zsum[s] += part[s];
+                                if (on) {
+                                    const int zpre = part[s] * (jj ? 1 : 2);   // weight 2^(1-jj)
+                                    uint16_t *slot = reinterpret_cast<uint16_t *>(
+                                        zp + ((s * 2 + k) * 16 + pair) * zs + gloc) + half;
+                                    *slot = static_cast<uint16_t>(zpre & 0xFFFF);
+                                }
+                            }
                         }
 #pragma unroll
                         for (int s = 0; s < kSlices; ++s) {
-                            zsum[s] += part[s];
-                            if (on) {
-                                const int zpre = part[s] * (jj ? 1 : 2);   // weight 2^(1-jj)
-                                uint16_t *slot = reinterpret_cast<uint16_t *>(
-                                    zp + ((s * 2 + k) * 16 + pair) * zs + gloc) + half;
-                                *slot = static_cast<uint16_t>(zpre & 0xFFFF);
-                            }
+                            zsum[s] += __shfl_xor_sync(0xffffffffu, zsum[s], 1);
+                            zsum[s] += __shfl_xor_sync(0xffffffffu, zsum[s], 2);
                         }
-                    }
+                        if (on && q == 0) {
 #pragma unroll
-                    for (int s = 0; s < kSlices; ++s) {
-                        zsum[s] += __shfl_xor_sync(0xffffffffu, zsum[s], 1);
-                        zsum[s] += __shfl_xor_sync(0xffffffffu, zsum[s], 2);
-                    }
-                    if (on && q == 0) {
-#pragma unroll
-                        for (int s = 0; s < kSlices; ++s) zinit[(s * 2 + k) * zs + gloc] = -zsum[s];
-                        // t = T * 2^-e and the accumulator ends at -T
-                        zscale[k * zs + gloc] = -__uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+                            for (int s = 0; s < kSlices; ++s) zinit[(s * 2 + k) * zs + gloc] = -zsum[s];
+                            // t = T * 2^-e and the accumulator ends at -T
+                            zscale[k * zs + gloc] = -__uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+                        }
                     }
                 }
             }
-            if (beta == 0)
-                for (int r = tid; r < prows; r += nthreads)
+            if (beta == 0) {
+                if (tid < prows) arow[tid] = apre;
+                for (int r = tid + nthreads; r < prows; r += nthreads)
                     arow[r] = make_float2(__ldg(p.a + pr0 + r), __ldg(p.a + p.N + pr0 + r));
+            }
             __syncthreads();
 
             // ---- rows: chunks of 32 groups across the warps of a row, groups of 8 rows along
@@ -414,6 +478,9 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     p.nchunks = nchunks;
     p.wpr = wpr;
     p.streams = streams;
+    const size_t xel = x_bf16 ? 2 : 4;
+    p.vec_x = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && ((static_cast<size_t>(ldx) * xel) % 16 == 0);
+    p.vec_b = (reinterpret_cast<uintptr_t>(b) % 16 == 0) && (K % 4 == 0);
 
     const uint32_t smem = bytes_for(pass_rows);
     auto kern = f32x ? gemv_kernel<true> : gemv_kernel<false>;
