@@ -23,10 +23,11 @@
 //    parallelism and no per-lane address work.  Before the programmatic-launch wait only L2
 //    prefetches are issued (of the block, of x, a and b): a prefetch returns no data to the
 //    SM, so it cannot observe a value the previous kernel on the stream is still writing.
-//  * Lane = 32-column group.  Warps split a row into chunks of 32 groups; each lane reads
-//    its group's word pair for 8 rows from shared memory and its z pairs per path, the
-//    bit-position loops run outside the row loop (8 independent accumulation chains), a
-//    butterfly sums the 8 rows over the lanes, and the chunk partials meet in shared memory.
+//  * Lane = 32-column group.  A work item is 8 rows x one chunk of 32 groups; items are
+//    dealt round-robin to the warps.  Each lane reads its group's word pair for the 8 rows
+//    and its 16 z-pair words per path (four 16-byte shared loads), runs 8 independent
+//    accumulation chains, a butterfly sums the 8 rows over the lanes, and the chunk
+//    partials meet in shared memory.
 //  * RABIT_F32 activations use two 15-bit slices of a 29-bit z (twice the dp2a work).
 #include <algorithm>
 
@@ -39,6 +40,10 @@ namespace {
 constexpr int kMaxThreads = 512;
 constexpr int kGroupRows = 8;            // rows per butterfly reduction and per copy barrier
 constexpr int kSmemBudget = 200 * 1024;  // dynamic shared memory a CTA may use
+// A group's 16 z-pair words per path and slice sit together, 20 words apart from the next
+// group's: a lane loads its own with four 16-byte reads, and the 8 lanes of a quarter warp
+// land on disjoint banks.
+constexpr int kZStride = 20;
 
 struct GemvArgs {
     const uint2 *packed;   // [N][Wr] groups {path-1 word, path-2 word}
@@ -52,8 +57,6 @@ struct GemvArgs {
     int rows_per_cta;      // contiguous rows owned by one CTA
     int pass_rows;         // rows staged in shared memory at a time (multiple of 8)
     int nchunks;           // 32-group chunks of a row
-    int wpr;               // warps across a row (each takes chunks wpr apart)
-    int streams;           // warps along rows
     int vec_x;             // x rows 16-byte aligned: 16-byte loads of 8 columns
     int vec_b;             // both b rows 16-byte aligned
 };
@@ -69,7 +72,7 @@ __host__ __device__ inline SmemLayout smem_layout(int pass_rows, int Wr, int nch
     uint32_t off = 0;
     auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 127u) & ~127u; return o; };
     L.w = take(static_cast<uint32_t>(pass_rows) * Wr * 8u);
-    L.zp = take(static_cast<uint32_t>(kSlices) * 2u * 16u * (Wr + 1) * 4u);
+    L.zp = take(static_cast<uint32_t>(kSlices) * 2u * Wr * kZStride * 4u);
     L.zinit = take(static_cast<uint32_t>(kSlices) * 2u * (Wr + 1) * 4u);
     L.zscale = take(2u * (Wr + 1) * 4u);
     L.arow = take(static_cast<uint32_t>(pass_rows) * 8u);
@@ -192,7 +195,7 @@ gemv_kernel(const GemvArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SmemLayout L = smem_layout<kSlices>(p.pass_rows, p.Wr, p.nchunks);
     uint2 *wbuf = reinterpret_cast<uint2 *>(smem + L.w);             // [pass_rows][Wr]
-    uint32_t *zp = reinterpret_cast<uint32_t *>(smem + L.zp);        // [slice][path][16][zs]
+    uint32_t *zp = reinterpret_cast<uint32_t *>(smem + L.zp);        // [slice][path][Wr][kZStride]
     int32_t *zinit = reinterpret_cast<int32_t *>(smem + L.zinit);    // [slice][path][zs]
     float *zscale = reinterpret_cast<float *>(smem + L.zscale);      // [path][zs]
     float2 *arow = reinterpret_cast<float2 *>(smem + L.arow);        // [pass_rows]
@@ -202,7 +205,7 @@ gemv_kernel(const GemvArgs p) {
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nthreads = blockDim.x;
-    const int wchunk = warp % p.wpr, stream = warp / p.wpr;
+    const int nwarps = nthreads >> 5;
     const int row_begin = blockIdx.x * p.rows_per_cta;
     const int row_end = min(p.N, row_begin + p.rows_per_cta);
     if (row_begin >= row_end) return;  // whole CTA, before any barrier
@@ -241,7 +244,6 @@ gemv_kernel(const GemvArgs p) {
     for (int pr0 = row_begin; pr0 < row_end; pr0 += p.pass_rows, parity ^= 1u) {
         const int prows = min(p.pass_rows, row_end - pr0);
         const int ngroups = (prows + kGroupRows - 1) / kGroupRows;
-        const int last_row = prows - 1;
         // ---- stage the pass's rows: one bulk copy per 8 rows, each on its own barrier
         if (warp == 0) {
             for (int g = lane; g < ngroups; g += 32) {
@@ -317,7 +319,7 @@ gemv_kernel(const GemvArgs p) {
                                 if (on) {
                                     const int zpre = part[s] * (jj ? 1 : 2);   // weight 2^(1-jj)
                                     uint16_t *slot = reinterpret_cast<uint16_t *>(
-                                        zp + ((s * 2 + k) * 16 + pair) * zs + gloc) + half;
+                                        zp + ((s * 2 + k) * p.Wr + gloc) * kZStride + pair) + half;
                                     *slot = static_cast<uint16_t>(zpre & 0xFFFF);
                                 }
                             }
@@ -338,90 +340,84 @@ gemv_kernel(const GemvArgs p) {
             }
             if (beta == 0) {
                 if (tid < prows) arow[tid] = apre;
-                for (int r = tid + nthreads; r < prows; r += nthreads)
-                    arow[r] = make_float2(__ldg(p.a + pr0 + r), __ldg(p.a + p.N + pr0 + r));
+                for (int r = tid + nthreads; r < p.pass_rows; r += nthreads)   // rows past prows: a = 0
+                    arow[r] = r < prows ? make_float2(__ldg(p.a + pr0 + r), __ldg(p.a + p.N + pr0 + r))
+                                        : make_float2(0.0f, 0.0f);
+                if (tid >= prows && tid < p.pass_rows) arow[tid] = make_float2(0.0f, 0.0f);
             }
             __syncthreads();
 
-            // ---- rows: chunks of 32 groups across the warps of a row, groups of 8 rows along
-            // the streams.
-            for (int c = wchunk; c < p.nchunks; c += p.wpr) {
+            // ---- rows: work items (8 rows x one 32-group chunk) dealt round-robin to the warps.
+            // Rows past prows in the last group read stale words of the pass buffer; their a is
+            // 0 and their totals are never stored.
+            const int nitems = ngroups * p.nchunks;
+            for (int item = warp; item < nitems; item += nwarps) {
+                const int g = item / p.nchunks;
+                const int c = item - g * p.nchunks;
                 const int gl = c * 32 + lane;
                 const bool lane_on = gl < p.Wr;
                 const int gz = lane_on ? gl : p.Wr - 1;     // lanes past the row read a valid word
-                int32_t init[kSlices][2];
-                float scl[2];
+                float sk[2];
+                if (beta == 0 && !mbar_wait_bounded(smem_u32(&bars[g]), parity, &abort_flag,
+                                                    p.timeout_ns, p.fault, FAULT_GEMV_WAIT_COPY))
+                    sk[0] = sk[1] = 0.0f;  // the copy never landed: contribute nothing
+                else
 #pragma unroll
-                for (int s = 0; s < kSlices; ++s)
+                    for (int k = 0; k < 2; ++k) sk[k] = lane_on ? zscale[k * zs + gz] : 0.0f;
+                uint2 w[kGroupRows];
+                const uint2 *wrow = wbuf + static_cast<int64_t>(g) * kGroupRows * p.Wr + gz;
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) init[s][k] = lane_on ? zinit[(s * 2 + k) * zs + gz] : 0;
+                for (int i = 0; i < kGroupRows; ++i) w[i] = wrow[static_cast<int64_t>(i) * p.Wr];
+                float tk[2][kGroupRows];
 #pragma unroll
-                for (int k = 0; k < 2; ++k) scl[k] = lane_on ? zscale[k * zs + gz] : 0.0f;
-
-                for (int g = stream; g < ngroups; g += p.streams) {
-                    if (beta == 0 && !mbar_wait_bounded(smem_u32(&bars[g]), parity, &abort_flag,
-                                                        p.timeout_ns, p.fault, FAULT_GEMV_WAIT_COPY))
-                        scl[0] = scl[1] = 0.0f;  // the copy never landed: contribute nothing
-                    uint2 w[kGroupRows];
+                for (int k = 0; k < 2; ++k) {
+                    int32_t acc[kSlices][kGroupRows];
+                    uint4 zq[kSlices][4];
 #pragma unroll
-                    for (int i = 0; i < kGroupRows; ++i)
-                        w[i] = wbuf[static_cast<int64_t>(min(g * kGroupRows + i, last_row)) * p.Wr + gz];
-                    float tk[2][kGroupRows];
-#pragma unroll 1
-                    for (int k = 0; k < 2; ++k) {
-                        uint32_t wk[kGroupRows];
+                    for (int s = 0; s < kSlices; ++s) {
+                        const uint4 *zrow = reinterpret_cast<const uint4 *>(zp + ((s * 2 + k) * p.Wr + gz) * kZStride);
 #pragma unroll
-                        for (int i = 0; i < kGroupRows; ++i) wk[i] = k ? w[i].y : w[i].x;
-                        int32_t acc[kSlices][kGroupRows];
+                        for (int j = 0; j < 4; ++j) zq[s][j] = zrow[j];
+                        const int32_t init = zinit[(s * 2 + k) * zs + gz];
 #pragma unroll
-                        for (int s = 0; s < kSlices; ++s)
+                        for (int i = 0; i < kGroupRows; ++i) acc[s][i] = init;
+                    }
+                    // bit positions 2sh and 2sh+1 of every byte; z pre-shifted to weigh them alike
 #pragma unroll
-                            for (int i = 0; i < kGroupRows; ++i) acc[s][i] = k ? init[s][1] : init[s][0];
-                        // one pair of bit positions per iteration; the bit-position loops sit
-                        // outside the row loop, so the 8 rows' chains overlap in the pipeline
-#pragma unroll 1
-                        for (int sh = 0; sh < 4; ++sh) {
-                            uint32_t zr[kSlices][4];
-#pragma unroll
-                            for (int s = 0; s < kSlices; ++s)
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) zr[s][i] = zp[((s * 2 + k) * 16 + sh * 4 + i) * zs + gz];
-#pragma unroll
-                            for (int jj = 0; jj < 2; ++jj) {
-#pragma unroll
-                                for (int i = 0; i < kGroupRows; ++i) {
-                                    const uint32_t bits = (wk[i] >> (2 * sh)) & (0x01010101u << jj);
-#pragma unroll
-                                    for (int s = 0; s < kSlices; ++s) {
-                                        uint32_t a0 = static_cast<uint32_t>(acc[s][i]);
-                                        a0 = dp2a_lo(zr[s][jj * 2 + 0], bits, a0);
-                                        a0 = dp2a_hi(zr[s][jj * 2 + 1], bits, a0);
-                                        acc[s][i] = static_cast<int32_t>(a0);
-                                    }
-                                }
-                            }
-                        }
-                        const float sk = k ? scl[1] : scl[0];
+                    for (int sh = 0; sh < 4; ++sh) {
 #pragma unroll
                         for (int i = 0; i < kGroupRows; ++i) {
-                            float t;
-                            if constexpr (kF32X)
-                                t = fmaf(static_cast<float>(acc[0][i]), 16384.0f, static_cast<float>(acc[1][i])) * sk;
-                            else
-                                t = static_cast<float>(acc[0][i]) * sk;
-                            if (k) tk[1][i] = t; else tk[0][i] = t;
+                            const uint32_t wv = (k ? w[i].y : w[i].x) >> (2 * sh);
+                            const uint32_t b0 = wv & 0x01010101u, b1 = wv & 0x02020202u;
+#pragma unroll
+                            for (int s = 0; s < kSlices; ++s) {
+                                uint32_t a0 = static_cast<uint32_t>(acc[s][i]);
+                                a0 = dp2a_lo(zq[s][sh].x, b0, a0);
+                                a0 = dp2a_hi(zq[s][sh].y, b0, a0);
+                                a0 = dp2a_lo(zq[s][sh].z, b1, a0);
+                                a0 = dp2a_hi(zq[s][sh].w, b1, a0);
+                                acc[s][i] = static_cast<int32_t>(a0);
+                            }
                         }
                     }
-                    float part[kGroupRows];
+                    // integer -> float by the 1.5 * 2^23 offset (|acc| < 2^22)
 #pragma unroll
                     for (int i = 0; i < kGroupRows; ++i) {
-                        const float2 av = arow[min(g * kGroupRows + i, last_row)];
-                        part[i] = fmaf(av.x, tk[0][i], av.y * tk[1][i]);
+                        float t = __int_as_float(acc[0][i] + 0x4B400000) - 12582912.0f;
+                        if constexpr (kF32X)
+                            t = fmaf(t, 16384.0f, __int_as_float(acc[1][i] + 0x4B400000) - 12582912.0f);
+                        tk[k][i] = t * sk[k];
                     }
-                    const float total = butterfly8(part, lane);
-                    const int ri = g * kGroupRows + ((lane >> 2) & 7);
-                    if ((lane & 3) == 0 && ri < prows) red[c * p.pass_rows + ri] = total;
                 }
+                float part[kGroupRows];
+#pragma unroll
+                for (int i = 0; i < kGroupRows; ++i) {
+                    const float2 av = arow[g * kGroupRows + i];
+                    part[i] = fmaf(av.x, tk[0][i], av.y * tk[1][i]);
+                }
+                const float total = butterfly8(part, lane);
+                const int ri = g * kGroupRows + ((lane >> 2) & 7);
+                if ((lane & 3) == 0 && ri < prows) red[c * p.pass_rows + ri] = total;
             }
             __syncthreads();
             // ---- y = sum of the chunk partials
@@ -444,7 +440,6 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
                         int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns) {
     const int Wr = static_cast<int>(padded_cols(K) / 32);
     const int nchunks = ceil_div(Wr, 32);
-    const int wpr = std::min(nchunks, kMaxThreads / 32);        // warps across a row
     // Rows: as evenly as possible over the SMs, one CTA each.
     const int rows_per_cta = ceil_div(N, std::min(ctx.num_sms, N));
     const int grid = ceil_div(N, rows_per_cta);
@@ -456,8 +451,9 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     while (pass_rows > kGroupRows && bytes_for(pass_rows) > static_cast<uint32_t>(kSmemBudget))
         pass_rows -= kGroupRows;
     if (bytes_for(pass_rows) > static_cast<uint32_t>(kSmemBudget)) return cudaErrorInvalidConfiguration;
-    const int streams = std::max(1, std::min(kMaxThreads / 32 / wpr, ceil_div(pass_rows, kGroupRows)));
-    const int threads = 32 * wpr * streams;
+    // one warp per work item of a pass (8 rows x 32 groups), at most kMaxThreads threads
+    const int items = ceil_div(pass_rows, kGroupRows) * nchunks;
+    const int threads = 32 * std::max(1, std::min(kMaxThreads / 32, items));
 
     GemvArgs p;
     p.packed = reinterpret_cast<const uint2 *>(packed);
@@ -476,8 +472,6 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     p.rows_per_cta = rows_per_cta;
     p.pass_rows = pass_rows;
     p.nchunks = nchunks;
-    p.wpr = wpr;
-    p.streams = streams;
     const size_t xel = x_bf16 ? 2 : 4;
     p.vec_x = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && ((static_cast<size_t>(ldx) * xel) % 16 == 0);
     p.vec_b = (reinterpret_cast<uintptr_t>(b) % 16 == 0) && (K % 4 == 0);
