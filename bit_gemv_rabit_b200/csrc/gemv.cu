@@ -10,13 +10,15 @@
 // Design for sm_100a (CUDA cores; the integer dot-product pipe sets the compute bound):
 //
 //  * Signs as masked sums.  t = Z - 2*sum_{bit=1} z with Z = sum_j z.  For each 32-column
-//    group z is quantised to 15-bit integers with a power-of-two scale of its own (the group
+//    group z is quantised to 13-bit integers with a power-of-two scale of its own (the group
 //    max fixes it, so the error is relative to the local maximum).  One 3-input logic op
-//    isolates four sign bits of a word at one position in each byte (values 0 or 2^q), and a
-//    dp2a multiplies two of those bytes with two pre-shifted 16-bit z values and accumulates
-//    in 32-bit: the integer sum is exact.  Two bit positions per byte (q in {0,1}) with z
-//    pre-shifted by 2^(1-q) give every product the same weight 2*z, so each path needs one
-//    accumulator, seeded with -Z.  Per 32 weight bits: 16 dp2a, 8 logic ops, 3 shifts.
+//    isolates four sign bits of a word at one position q in each byte (values 0 or 2^q),
+//    and a dp2a multiplies two of those bytes with two pre-shifted 16-bit z values and
+//    accumulates in 32-bit: the integer sum is exact.  Four bit positions per byte
+//    (q = 0..3, then the word shifted by 4) with z pre-shifted by 2^(3-q) give every product
+//    the same weight 8*z, so each path needs one accumulator, seeded with -4Z.  Per 32
+//    weight bits: 16 dp2a (the fma-heavy pipe, which bounds the kernel), 8 logic ops and
+//    one shift.
 //  * A CTA owns a contiguous block of whole rows, which is one contiguous range of the
 //    row-major packed layout: TMA bulk copies (one per 8 rows, each completing on its own
 //    mbarrier) bring it into shared memory, so the weight stream has deep memory-level
@@ -28,7 +30,7 @@
 //    and its 16 z-pair words per path (four 16-byte shared loads), runs 8 independent
 //    accumulation chains, a butterfly sums the 8 rows over the lanes, and the chunk
 //    partials meet in shared memory.
-//  * RABIT_F32 activations use two 15-bit slices of a 29-bit z (twice the dp2a work).
+//  * RABIT_F32 activations use two 13-bit slices of a 24-bit z (twice the dp2a work).
 #include <algorithm>
 
 #include "rabit_device.cuh"
@@ -37,7 +39,7 @@
 namespace rabit {
 namespace {
 
-constexpr int kMaxThreads = 512;
+constexpr int kMaxThreads = 768;
 constexpr int kGroupRows = 8;            // rows per butterfly reduction and per copy barrier
 constexpr int kSmemBudget = 200 * 1024;  // dynamic shared memory a CTA may use
 // A group's 16 z-pair words per path and slice sit together, 20 words apart from the next
@@ -290,11 +292,11 @@ gemv_kernel(const GemvArgs p) {
                         }
                         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
                         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                        // power-of-two scale 2^e with m * 2^e <= kMaxQ (15-bit, or 29-bit for fp32 x)
-                        constexpr int kTop = kF32X ? 27 : 13;
-                        const float kMaxQ = kF32X ? 268435455.0f : 16383.0f;
+                        // power-of-two scale 2^e with m * 2^e <= kMaxQ (13-bit, or 24-bit for fp32 x)
+                        constexpr int kTop = kF32X ? 22 : 11;
+                        const float kMaxQ = kF32X ? 8388607.0f : 4095.0f;
                         const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xFFu) - 127;
-                        int e = min(127, max(-126, kTop - E));
+                        int e = min(124, max(-126, kTop - E));
                         float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
                         if (m * sc > kMaxQ) { --e; sc *= 0.5f; }
                         int zsum[kSlices];
@@ -302,13 +304,15 @@ gemv_kernel(const GemvArgs p) {
                         for (int s = 0; s < kSlices; ++s) zsum[s] = 0;
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const int sh = i >> 1, jj = i & 1;
-                            const int pair = sh * 4 + jj * 2 + h;
+                            // column 8q+i sits at bit i of byte q: bit position i&3 after a shift
+                            // by 4*(i>>2); dp2a.lo takes bytes 0,1 and dp2a.hi bytes 2,3
+                            const int qb = i & 3;
+                            const int pair = (i >> 2) * 8 + qb * 2 + h;
                             int part[kSlices];
                             if constexpr (kF32X) {
                                 const int zq = __float2int_rn(zv[u][k][i] * sc);
-                                part[0] = (zq + (1 << 13)) >> 14;       // high 15-bit slice
-                                part[1] = zq - (part[0] << 14);         // low slice, in [-2^13, 2^13)
+                                part[0] = (zq + (1 << 11)) >> 12;       // high 13-bit slice
+                                part[1] = zq - (part[0] << 12);         // low slice, in [-2^11, 2^11)
                             } else {
                                 // round to nearest even by adding 1.5 * 2^23 (|z * 2^e| < 2^22)
                                 part[0] = __float_as_int(fmaf(zv[u][k][i], sc, 12582912.0f)) - 0x4B400000;
@@ -317,7 +321,7 @@ gemv_kernel(const GemvArgs p) {
                             for (int s = 0; s < kSlices; ++s) {
                                 zsum[s] += part[s];
                                 if (on) {
-                                    const int zpre = part[s] * (jj ? 1 : 2);   // weight 2^(1-jj)
+                                    const int zpre = part[s] << (3 - qb);      // weight 2^(3-q)
                                     uint16_t *slot = reinterpret_cast<uint16_t *>(
                                         zp + ((s * 2 + k) * p.Wr + gloc) * kZStride + pair) + half;
                                     *slot = static_cast<uint16_t>(zpre & 0xFFFF);
@@ -331,9 +335,9 @@ gemv_kernel(const GemvArgs p) {
                         }
                         if (on && q == 0) {
 #pragma unroll
-                            for (int s = 0; s < kSlices; ++s) zinit[(s * 2 + k) * zs + gloc] = -zsum[s];
-                            // t = T * 2^-e and the accumulator ends at -T
-                            zscale[k * zs + gloc] = -__uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+                            for (int s = 0; s < kSlices; ++s) zinit[(s * 2 + k) * zs + gloc] = -4 * zsum[s];
+                            // the accumulator ends at -4T and t = T * 2^-e
+                            zscale[k * zs + gloc] = -__uint_as_float(static_cast<uint32_t>(125 - e) << 23);
                         }
                     }
                 }
@@ -351,9 +355,10 @@ gemv_kernel(const GemvArgs p) {
             // Rows past prows in the last group read stale words of the pass buffer; their a is
             // 0 and their totals are never stored.
             const int nitems = ngroups * p.nchunks;
+            // (g, c) of item warp + j * nwarps, advanced without a division per item
+            const int gstep = nwarps / p.nchunks, cstep = nwarps - gstep * p.nchunks;
+            int g = warp / p.nchunks, c = warp - (warp / p.nchunks) * p.nchunks;
             for (int item = warp; item < nitems; item += nwarps) {
-                const int g = item / p.nchunks;
-                const int c = item - g * p.nchunks;
                 const int gl = c * 32 + lane;
                 const bool lane_on = gl < p.Wr;
                 const int gz = lane_on ? gl : p.Wr - 1;     // lanes past the row read a valid word
@@ -382,42 +387,49 @@ gemv_kernel(const GemvArgs p) {
 #pragma unroll
                         for (int i = 0; i < kGroupRows; ++i) acc[s][i] = init;
                     }
-                    // bit positions 2sh and 2sh+1 of every byte; z pre-shifted to weigh them alike
+                    // bit position q of every byte (after a shift by 0 or 4) has the value 2^q;
+                    // z is pre-shifted by 2^(3-q), so every product weighs 8 z
 #pragma unroll
-                    for (int sh = 0; sh < 4; ++sh) {
+                    for (int s4 = 0; s4 < 2; ++s4) {
 #pragma unroll
                         for (int i = 0; i < kGroupRows; ++i) {
-                            const uint32_t wv = (k ? w[i].y : w[i].x) >> (2 * sh);
-                            const uint32_t b0 = wv & 0x01010101u, b1 = wv & 0x02020202u;
+                            const uint32_t wv = (k ? w[i].y : w[i].x) >> (4 * s4);
 #pragma unroll
                             for (int s = 0; s < kSlices; ++s) {
                                 uint32_t a0 = static_cast<uint32_t>(acc[s][i]);
-                                a0 = dp2a_lo(zq[s][sh].x, b0, a0);
-                                a0 = dp2a_hi(zq[s][sh].y, b0, a0);
-                                a0 = dp2a_lo(zq[s][sh].z, b1, a0);
-                                a0 = dp2a_hi(zq[s][sh].w, b1, a0);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const uint32_t bq = wv & (0x01010101u << q);
+                                    const uint4 &zz = zq[s][s4 * 2 + (q >> 1)];
+                                    a0 = dp2a_lo((q & 1) ? zz.z : zz.x, bq, a0);
+                                    a0 = dp2a_hi((q & 1) ? zz.w : zz.y, bq, a0);
+                                }
                                 acc[s][i] = static_cast<int32_t>(a0);
                             }
                         }
                     }
-                    // integer -> float by the 1.5 * 2^23 offset (|acc| < 2^22)
+                    // |acc| < 2^21: the conversions are exact
 #pragma unroll
                     for (int i = 0; i < kGroupRows; ++i) {
-                        float t = __int_as_float(acc[0][i] + 0x4B400000) - 12582912.0f;
-                        if constexpr (kF32X)
-                            t = fmaf(t, 16384.0f, __int_as_float(acc[1][i] + 0x4B400000) - 12582912.0f);
+                        float t = static_cast<float>(acc[0][i]);
+                        if constexpr (kF32X) t = fmaf(t, 4096.0f, static_cast<float>(acc[1][i]));
                         tk[k][i] = t * sk[k];
                     }
                 }
                 float part[kGroupRows];
+                const float4 *a4 = reinterpret_cast<const float4 *>(arow + g * kGroupRows);
 #pragma unroll
-                for (int i = 0; i < kGroupRows; ++i) {
-                    const float2 av = arow[g * kGroupRows + i];
-                    part[i] = fmaf(av.x, tk[0][i], av.y * tk[1][i]);
+                for (int i = 0; i < kGroupRows / 2; ++i) {
+                    const float4 av = a4[i];
+                    part[2 * i] = fmaf(av.x, tk[0][2 * i], av.y * tk[1][2 * i]);
+                    part[2 * i + 1] = fmaf(av.z, tk[0][2 * i + 1], av.w * tk[1][2 * i + 1]);
                 }
                 const float total = butterfly8(part, lane);
                 const int ri = g * kGroupRows + ((lane >> 2) & 7);
                 if ((lane & 3) == 0 && ri < prows) red[c * p.pass_rows + ri] = total;
+                g += gstep;
+                c += cstep;
+                if (c >= p.nchunks) { c -= p.nchunks; ++g; }
             }
             __syncthreads();
             // ---- y = sum of the chunk partials
@@ -451,9 +463,14 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     while (pass_rows > kGroupRows && bytes_for(pass_rows) > static_cast<uint32_t>(kSmemBudget))
         pass_rows -= kGroupRows;
     if (bytes_for(pass_rows) > static_cast<uint32_t>(kSmemBudget)) return cudaErrorInvalidConfiguration;
-    // one warp per work item of a pass (8 rows x 32 groups), at most kMaxThreads threads
+    // Warps: as few as give every warp the same number of work items (8 rows x 32 groups)
+    // within kMaxThreads, but enough that the z stage has at most two tasks per thread
+    // (up to 16 warps).
     const int items = ceil_div(pass_rows, kGroupRows) * nchunks;
-    const int threads = 32 * std::max(1, std::min(kMaxThreads / 32, items));
+    const int max_warps = kMaxThreads / 32;
+    const int per_warp = ceil_div(items, max_warps);
+    const int zwarps = std::min(16, ceil_div(4 * Wr, 64));
+    const int threads = 32 * std::min(max_warps, std::max(ceil_div(items, per_warp), zwarps));
 
     GemvArgs p;
     p.packed = reinterpret_cast<const uint2 *>(packed);
