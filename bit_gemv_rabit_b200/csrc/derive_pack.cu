@@ -7,12 +7,15 @@
 // RABIT_LAYOUT_V2 arrangement declared in include/rabit.h.
 //
 // HBM-bound: W is streamed once (4 or 2 bytes per weight), 2 bits per weight are written.
-// One warp handles one row and 32 consecutive 32-column groups of it (1024 columns): in
-// step i lane l reads column 32*(w0+i) + l (128 contiguous bytes per warp load for fp32 W),
-// forms both signs, and __ballot_sync turns the 32 lanes' signs into one packed word, so the
-// bit order (column j -> bit j % 32) falls out of the lane order.  Lane i keeps the word
-// pair of step i, and the warp then stores its 32 uint2 groups with one coalesced 256-byte
-// store.  R1 is never stored.
+// A warp owns one 1024-column chunk (32 groups) and walks rows: it keeps the chunk's b
+// values in registers, and in step i lane l reads column 32*(w0+i) + l of the row (128
+// contiguous bytes per warp load for fp32 W), forms both signs, and __ballot_sync turns the
+// 32 lanes' signs into one packed word, so the bit order (column j -> bit j % 32) falls out
+// of the lane order.  Lane 0 parks the word pair of step i in shared memory, and the warp
+// then stores the row's 32 uint2 groups with one coalesced 256-byte store.  Chunks wholly
+// inside the row skip the column bound checks.  R1 is never stored.
+#include <algorithm>
+
 #include "rabit_device.cuh"
 #include "rabit_kernels.h"
 
@@ -31,52 +34,67 @@ __device__ __forceinline__ float load_w(const void *W, int64_t idx) {
     }
 }
 
+// Signs of 32 columns (one per lane) of row n for step i of a task; the ballots make the two
+// packed words, and lane 0 parks them in the warp's shared slot i.
+template <bool kFull>
+__device__ __forceinline__ void derive_step(float w, float b1, float a1, bool ok, int i, uint2 *slots, int lane) {
+    const bool neg1 = w < 0.0f;                                  // S1 = sign(W)
+    // R1 = W - a1*S1*b1 with a single rounding: the sign of R1 is exact.
+    const float r1 = fmaf(neg1 ? a1 : -a1, b1, w);
+    const bool neg2 = r1 < 0.0f;                                 // S2 = sign(R1)
+    const uint32_t s1w = __ballot_sync(0xffffffffu, kFull ? neg1 : (ok && neg1));
+    const uint32_t s2w = __ballot_sync(0xffffffffu, kFull ? neg2 : (ok && neg2));
+    if (lane == 0) slots[i] = make_uint2(s1w, s2w);
+}
+
 template <bool kBf16>
 __global__ void __launch_bounds__(kDeriveThreads)
 derive_pack_kernel(const void *__restrict__ W, int N, int K, int ldw,
                    const float *__restrict__ a, const float *__restrict__ b,
                    uint2 *__restrict__ packed, int Wr) {
+    __shared__ uint2 slot_buf[kDeriveThreads / 32][32];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
     const int lane = threadIdx.x & 31;
+    uint2 *slots = slot_buf[threadIdx.x >> 5];
     const int chunks = (Wr + 31) / 32;  // 1024-column chunks per row
-    const int64_t num_tasks = static_cast<int64_t>(N) * chunks;
-    const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kDeriveThreads + threadIdx.x) >> 5;
-    const int64_t warp_stride = (static_cast<int64_t>(gridDim.x) * kDeriveThreads) >> 5;
+    // The launch makes the warp count a multiple of `chunks`, so a warp keeps one chunk (and
+    // its b values) for all the rows it visits.
+    const int warp_global = (blockIdx.x * kDeriveThreads + threadIdx.x) >> 5;
+    const int warps = (gridDim.x * kDeriveThreads) >> 5;
+    const int chunk = warp_global % chunks;
+    const int w0 = chunk * 32;
+    const bool full = (w0 + 32) * 32 <= K;   // every column of the chunk is inside the row
 
-    for (int64_t task = warp_global; task < num_tasks; task += warp_stride) {
-        const int n = static_cast<int>(task / chunks);
-        const int w0 = static_cast<int>(task % chunks) * 32;
+    float b1[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int j = (w0 + i) * 32 + lane;
+        b1[i] = j < K ? __ldg(b + j) : 0.0f;
+    }
+    for (int n = warp_global / chunks; n < N; n += warps / chunks) {
         const float a1 = __ldg(a + n);
         const int64_t row = static_cast<int64_t>(n) * ldw;
-
-        float w[32], b1[32];
+        float w[32];
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int j = (w0 + i) * 32 + lane;
-            const bool ok = j < K;
-            w[i] = ok ? load_w<kBf16>(W, row + j) : 0.0f;
-            b1[i] = ok ? __ldg(b + j) : 0.0f;
-        }
-        uint32_t mine1 = 0, mine2 = 0;
+            for (int i = 0; i < 32; ++i) w[i] = load_w<kBf16>(W, row + (w0 + i) * 32 + lane);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int j = (w0 + i) * 32 + lane;
-            const bool ok = j < K;
-            const bool neg1 = w[i] < 0.0f;                          // S1 = sign(W)
-            // R1 = W - a1*S1*b1 with a single rounding: the sign of R1 is exact.
-            const float r1 = fmaf(neg1 ? a1 : -a1, b1[i], w[i]);
-            const bool neg2 = r1 < 0.0f;                            // S2 = sign(R1)
-            const uint32_t s1w = __ballot_sync(0xffffffffu, ok && neg1);
-            const uint32_t s2w = __ballot_sync(0xffffffffu, ok && neg2);
-            if (lane == i) {
-                mine1 = s1w;
-                mine2 = s2w;
+            for (int i = 0; i < 32; ++i) derive_step<true>(w[i], b1[i], a1, true, i, slots, lane);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int j = (w0 + i) * 32 + lane;
+                w[i] = j < K ? load_w<kBf16>(W, row + j) : 0.0f;
             }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                derive_step<false>(w[i], b1[i], a1, (w0 + i) * 32 + lane < K, i, slots, lane);
         }
-        if (w0 + lane < Wr)
-            packed[static_cast<int64_t>(n) * Wr + w0 + lane] = make_uint2(mine1, mine2);
+        __syncwarp();
+        if (w0 + lane < Wr) packed[static_cast<int64_t>(n) * Wr + w0 + lane] = slots[lane];
+        __syncwarp();
     }
 }
 
@@ -85,11 +103,16 @@ derive_pack_kernel(const void *__restrict__ W, int N, int K, int ldw,
 cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16, int N, int K,
                                int ldw, const float *a, const float *b, uint32_t *packed) {
     const int Wr = static_cast<int>(padded_cols(K) / 32);
-    const int64_t tasks = static_cast<int64_t>(N) * ((Wr + 31) / 32);
+    // Warps: a multiple of the chunk count (so each warp keeps one chunk), enough for every
+    // (row, chunk) task when there are few, at most 8 CTAs per SM.
+    const int chunks = (Wr + 31) / 32;
     const int64_t warps_per_block = kDeriveThreads / 32;
-    int64_t blocks = (tasks + warps_per_block - 1) / warps_per_block;
-    const int64_t max_blocks = static_cast<int64_t>(ctx.num_sms) * 8;
-    if (blocks > max_blocks) blocks = max_blocks;
+    const int64_t want = std::min<int64_t>(static_cast<int64_t>(N) * chunks,
+                                           static_cast<int64_t>(ctx.num_sms) * 8 * warps_per_block);
+    int64_t warps = std::max<int64_t>(chunks, (want / chunks) * chunks);
+    // round up to whole blocks while keeping a multiple of chunks
+    while (warps % warps_per_block != 0) warps += chunks;
+    const int64_t blocks = warps / warps_per_block;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));

@@ -1,0 +1,71 @@
+"""A device wait that runs out is reported, not hung on.
+
+The GEMM's test switch RABIT_TEST_SKIP_ONE_ARRIVE makes the expansion warps skip their first
+arrival, so the MMA warp's bounded wait on that stage expires (after RABIT_WAIT_TIMEOUT_MS).
+The kernel then drains its in-flight copies, frees tensor memory and returns; the host reads
+RABIT_ERR_TIMEOUT with the wait's fault bit, and the next call on the same context is
+correct.  No GPU fault is involved: the failure is a missing arrival that a flag withholds.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_gemv_rabit_b200 import inputs
+from bit_gemv_rabit_b200 import rabit
+
+pytestmark = pytest.mark.gpu
+
+FAULT_GEMM_WAIT_MMA = 1 << 1
+RABIT_ERR_TIMEOUT = -8
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from bit_gemv_rabit_b200 import build
+    build.build()
+    rabit.load()
+    rabit.rabit_read_fault(clear=True)
+    yield
+    assert rabit.rabit_read_fault(clear=True) == 0
+
+
+def _case(N=256, K=512, M=256, seed=4242):
+    W = inputs.weight(seed, N, K)
+    a, b = inputs.scales(seed, W)
+    x = inputs.activations(seed, M, K)
+    dev = lambda v: torch.from_numpy(np.ascontiguousarray(v)).cuda()
+    at, bt = dev(a), dev(b)
+    packed = rabit.alloc_packed(N, K)
+    rabit.rabit_derive_pack(dev(W), at, bt, packed)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    return W, a, b, x, at, bt, packed, xt
+
+
+def test_gemm_wait_expiry_is_reported_and_the_context_survives(monkeypatch):
+    N, K, M = 256, 512, 256
+    W, a, b, x, at, bt, packed, xt = _case(N, K, M)
+    ws = rabit.alloc_gemm_workspace(N, K, 2, M)
+    y = torch.zeros((M, N), device="cuda")
+    monkeypatch.setenv("RABIT_TEST_SKIP_ONE_ARRIVE", "1")
+    monkeypatch.setenv("RABIT_WAIT_TIMEOUT_MS", "50")
+    rabit.rabit_gemm(packed, at, bt, N, K, xt, y, ws)
+    flags = ctypes.c_uint32(0)
+    st = rabit.load().rabit_read_fault(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
+                                        ctypes.byref(flags), 1)
+    assert st == RABIT_ERR_TIMEOUT
+    assert flags.value & FAULT_GEMM_WAIT_MMA
+    monkeypatch.delenv("RABIT_TEST_SKIP_ONE_ARRIVE")
+    monkeypatch.delenv("RABIT_WAIT_TIMEOUT_MS")
+    # the same context runs the same call correctly afterwards
+    rabit.rabit_gemm(packed, at, bt, N, K, xt, y, ws)
+    torch.cuda.synchronize()
+    assert rabit.rabit_read_fault(clear=True) == 0
+    S = oracle.derive_signs(W, a, b)
+    ref = oracle.layer(S, a, b, x)
+    err = float(np.max(np.abs(y.cpu().numpy() - ref)) / np.max(np.abs(ref)))
+    assert err <= 2e-3
