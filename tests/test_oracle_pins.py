@@ -304,3 +304,70 @@ def test_bf16_weight_widens_exactly():
     S_bits = oracle.derive_signs(Wb, a, b)
     S_f32 = oracle.derive_signs(inputs.bf16_to_f32(Wb), a, b)
     np.testing.assert_array_equal(S_bits, S_f32)
+
+
+# ---- three paths: the residual rule applied once more (S_3 = sign(W - W_hat_1 - W_hat_2)),
+# grouped as three words plus a zero padding word (Appendix E.1 "Weight Packing", PackedBits3).
+
+def _three_path_layer(seed, N, K):
+    W = inputs.weight(seed, N, K)
+    a, b = inputs.scales(seed, W, P=3)
+    return W, a, b
+
+
+def test_three_path_signs_follow_the_residual_rule():
+    # brute force per element on a small case, written out in float64 here
+    rng = np.random.default_rng(71)
+    N, K = 8, 24
+    W = rng.standard_normal((N, K)).astype(F32)
+    a = rng.uniform(0.1, 0.9, (3, N)).astype(F32)
+    b = rng.uniform(0.1, 0.9, (3, K)).astype(F32)
+    S = oracle.derive_signs(W, a, b, P=3)
+    S2 = oracle.derive_signs(W, a, b, P=2)
+    np.testing.assert_array_equal(S[:2], S2)          # the first two paths do not change
+    for n in range(N):
+        for j in range(K):
+            r = float(W[n, j])
+            for k in range(3):
+                c = float(a[k, n]) * float(b[k, j])
+                errs = {s: (r - c * s) ** 2 for s in (+1, -1)}
+                best = +1 if errs[+1] <= errs[-1] else -1
+                assert S[k, n, j] == best
+                r -= c * best
+
+
+def test_three_path_frobenius_identity_and_hierarchy():
+    W, a, b = _three_path_layer(72, 48, 160)
+    S = oracle.derive_signs(W, a, b, P=3)
+    Wd = W.astype(np.float64)
+    c = [np.outer(a[k].astype(np.float64), b[k].astype(np.float64)) for k in range(3)]
+    W2 = c[0] * S[0] + c[1] * S[1]
+    W3 = W2 + c[2] * S[2]
+    R2 = Wd - W2
+    lhs = np.sum((Wd - W3) ** 2)
+    rhs = np.sum(R2 ** 2) - 2 * np.sum(c[2] * np.abs(R2)) + np.sum(c[2] ** 2)
+    assert lhs == pytest.approx(rhs, rel=1e-12)
+    assert np.linalg.norm(Wd - W3) <= np.linalg.norm(Wd - W2)
+
+
+def test_three_path_pack_groups_and_roundtrip():
+    rng = np.random.default_rng(73)
+    N, K = 5, 200                                      # Kp = 256: 8 groups of 4 words per row
+    S = np.where(rng.random((3, N, K)) < 0.5, -1, 1).astype(np.int8)
+    packed = oracle.pack(S)
+    assert packed.size == N * 8 * 4
+    np.testing.assert_array_equal(oracle.unpack(packed, N, K, P=3), S)
+    assert np.all(packed.reshape(N, 8, 4)[:, :, 3] == 0)    # the padding word of every group
+    # hand check: path 3 (k=2), row 4, column 37 -> word (4*8 + 1)*4 + 2 = 134, bit 5
+    S1 = np.ones((3, N, K), dtype=np.int8)
+    S1[2, 4, 37] = -1
+    p1 = oracle.pack(S1)
+    assert p1[134] == 1 << 5 and np.count_nonzero(p1) == 1
+
+
+def test_three_path_layer_matches_numpy_matmul():
+    W, a, b = _three_path_layer(74, 40, 130)
+    S = oracle.derive_signs(W, a, b, P=3)
+    x = inputs.bf16_to_f32(inputs.activations(74, 3, 130)).astype(np.float64)
+    W_hat = sum(np.outer(a[k].astype(np.float64), b[k].astype(np.float64)) * S[k] for k in range(3))
+    np.testing.assert_allclose(oracle.layer(S, a, b, x), x @ W_hat.T, rtol=1e-12, atol=1e-14)
