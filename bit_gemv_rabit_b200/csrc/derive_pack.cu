@@ -98,10 +98,55 @@ derive_pack_kernel(const void *__restrict__ W, int N, int K, int ldw,
     }
 }
 
+// Three paths (the residual rule once more: S3 = sign(W - W_hat_1 - W_hat_2)), groups of
+// three words plus a zero padding word.  The second residual needs the first one's value,
+// not only its sign, so both are formed in binary64 exactly as the definition reads: each
+// product a*s*b of two fp32 numbers is exact in binary64 and each subtraction rounds once.
+template <bool kBf16>
+__global__ void __launch_bounds__(kDeriveThreads)
+derive_pack3_kernel(const void *__restrict__ W, int N, int K, int ldw,
+                    const float *__restrict__ a, const float *__restrict__ b,
+                    uint4 *__restrict__ packed, int Wr) {
+    __shared__ uint4 slot_buf[kDeriveThreads / 32][32];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const int lane = threadIdx.x & 31;
+    uint4 *slots = slot_buf[threadIdx.x >> 5];
+    const int chunks = (Wr + 31) / 32;
+    const int warp_global = (blockIdx.x * kDeriveThreads + threadIdx.x) >> 5;
+    const int warps = (gridDim.x * kDeriveThreads) >> 5;
+    const int chunk = warp_global % chunks;
+    const int w0 = chunk * 32;
+    for (int n = warp_global / chunks; n < N; n += warps / chunks) {
+        const double a1 = __ldg(a + n), a2 = __ldg(a + N + n);   // S3 needs no third scale
+        const int64_t row = static_cast<int64_t>(n) * ldw;
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+            const int j = (w0 + i) * 32 + lane;
+            const bool ok = j < K;
+            const double w = ok ? static_cast<double>(load_w<kBf16>(W, row + j)) : 0.0;
+            const double b1 = ok ? __ldg(b + j) : 0.0, b2 = ok ? __ldg(b + K + j) : 0.0;
+            const bool neg1 = w < 0.0;
+            const double r1 = __dsub_rn(w, __dmul_rn(__dmul_rn(a1, neg1 ? -1.0 : 1.0), b1));
+            const bool neg2 = r1 < 0.0;
+            const double r2 = __dsub_rn(r1, __dmul_rn(__dmul_rn(a2, neg2 ? -1.0 : 1.0), b2));
+            const bool neg3 = r2 < 0.0;
+            const uint32_t s1w = __ballot_sync(0xffffffffu, ok && neg1);
+            const uint32_t s2w = __ballot_sync(0xffffffffu, ok && neg2);
+            const uint32_t s3w = __ballot_sync(0xffffffffu, ok && neg3);
+            if (lane == 0) slots[i] = make_uint4(s1w, s2w, s3w, 0u);
+        }
+        __syncwarp();
+        if (w0 + lane < Wr) packed[static_cast<int64_t>(n) * Wr + w0 + lane] = slots[lane];
+        __syncwarp();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16, int N, int K,
-                               int ldw, const float *a, const float *b, uint32_t *packed) {
+                               int ldw, int P, const float *a, const float *b, uint32_t *packed) {
     const int Wr = static_cast<int>(padded_cols(K) / 32);
     // Warps: a multiple of the chunk count (so each warp keeps one chunk), enough for every
     // (row, chunk) task when there are few, at most 8 CTAs per SM.
@@ -124,6 +169,12 @@ cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16,
     attr[0].val.programmaticStreamSerializationAllowed = ctx.pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (P == 3) {
+        uint4 *out3 = reinterpret_cast<uint4 *>(packed);
+        if (w_bf16)
+            return cudaLaunchKernelEx(&cfg, derive_pack3_kernel<true>, W, N, K, ldw, a, b, out3, Wr);
+        return cudaLaunchKernelEx(&cfg, derive_pack3_kernel<false>, W, N, K, ldw, a, b, out3, Wr);
+    }
     uint2 *out = reinterpret_cast<uint2 *>(packed);
     if (w_bf16)
         return cudaLaunchKernelEx(&cfg, derive_pack_kernel<true>, W, N, K, ldw, a, b, out, Wr);

@@ -77,6 +77,7 @@ __device__ __forceinline__ uint32_t half_bits(float v) {
     return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v)));
 }
 
+template <int kP>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -86,7 +87,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kblocks_per_path = p.Kp / kBK;
-    const int nkb = 2 * kblocks_per_path;
+    const int nkb = kP * kblocks_per_path;
     volatile int *abort_flag = &ctl->abort;
 
     if (threadIdx.x == 0) {
@@ -133,8 +134,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
                     }
                     const uint32_t bar = smem_u32(&ctl->full_b[s]);
                     mbar_arrive_expect_tx(bar, kStageBytes);
-                    const int path = kb & 1;            // K blocks alternate between the paths
-                    const int kcol = (kb >> 1) * kBK;
+                    const int path = kb % kP;           // K blocks cycle through the paths
+                    const int kcol = (kb / kP) * kBK;
                     tma_load_3d(smem_u32(smem + s * kStageBytes), &tmap_x, bar, kcol, m0, path);
                     issued[s] = true;
                     last_parity[s] = ph;
@@ -208,30 +209,48 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
             const int n0 = (tile / p.tiles_m) * kBM;
             const int n = n0 + row;
             const bool row_valid = n < p.N;
-            uint32_t a2[2];
+            uint32_t a2[kP];
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
+            for (int k = 0; k < kP; ++k) {
                 const uint32_t h = row_valid ? half_bits(__ldg(p.a + k * p.N + n)) : 0u;
                 a2[k] = h | (h << 16);
             }
-            // One 16-byte load gives both paths' words of a 64-column block:
-            // {path1 w, path2 w, path1 w+1, path2 w+1} with w = 2*block.
-            const uint4 *row_ptr = reinterpret_cast<const uint4 *>(p.packed + static_cast<int64_t>(n) * Wr * 2);
-            auto load_block = [&](int blk) -> uint4 {
-                return row_valid ? __ldg(row_ptr + blk) : make_uint4(0u, 0u, 0u, 0u);
+            // The packed words of one 64-column block (two 32-column groups) of this row:
+            // two paths: one 16-byte load {path1 w, path2 w, path1 w+1, path2 w+1};
+            // three paths: two 16-byte loads {path1, path2, path3, pad} of groups w and w+1.
+            struct Block { uint4 g0, g1; };
+            constexpr int kGroupWords = kP == 2 ? 2 : 4;     // words per 32-column group
+            const uint4 *row_ptr = reinterpret_cast<const uint4 *>(p.packed + static_cast<int64_t>(n) * Wr * kGroupWords);
+            auto load_block = [&](int blk) -> Block {
+                Block r{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+                if (row_valid) {
+                    if constexpr (kP == 2) {
+                        r.g0 = __ldg(row_ptr + blk);
+                    } else {
+                        r.g0 = __ldg(row_ptr + 2 * blk);
+                        r.g1 = __ldg(row_ptr + 2 * blk + 1);
+                    }
+                }
+                return r;
             };
-            uint4 cur = load_block(0);
-            uint4 nxt = nkb > 2 ? load_block(1) : make_uint4(0u, 0u, 0u, 0u);
+            Block cur = load_block(0);
+            Block nxt = kblocks_per_path > 1 ? load_block(1) : Block{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
-                const int path = kb & 1;
-                const uint32_t wlo = path ? cur.y : cur.x;   // columns [64*blk, 64*blk + 32)
-                const uint32_t whi = path ? cur.w : cur.z;   // columns [64*blk + 32, 64*blk + 64)
-                const uint32_t amag = path ? a2[1] : a2[0];
-                if (path) {
+                const int path = kb % kP;
+                uint32_t wlo, whi;                               // columns [64 blk, +32) and [+32, +64)
+                if constexpr (kP == 2) {
+                    wlo = path ? cur.g0.y : cur.g0.x;
+                    whi = path ? cur.g0.w : cur.g0.z;
+                } else {
+                    wlo = path == 0 ? cur.g0.x : (path == 1 ? cur.g0.y : cur.g0.z);
+                    whi = path == 0 ? cur.g1.x : (path == 1 ? cur.g1.y : cur.g1.z);
+                }
+                const uint32_t amag = path == 0 ? a2[0] : (path == 1 ? a2[1] : a2[kP - 1]);
+                if (path == kP - 1) {
                     cur = nxt;
-                    const int nb = (kb >> 1) + 2;
-                    if (2 * nb < nkb) nxt = load_block(nb);
+                    const int nb = kb / kP + 2;
+                    if (nb < kblocks_per_path) nxt = load_block(nb);
                 }
                 uint32_t v[32];
 #pragma unroll
@@ -290,14 +309,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
 }
 
 // X'_k[m][32g + 2c + h] = fp16(x[m][32g + c + 16h] * b_k[32g + c + 16h]) for c < 16,
-// 0 beyond K.  Layout [2][M][Kp]; one thread writes one (c, c+16) pair as a 32-bit word.
+// 0 beyond K.  Layout [P][M][Kp]; one thread writes one (c, c+16) pair as a 32-bit word.
 __global__ void __launch_bounds__(256)
 prep_x_kernel(const uint16_t *__restrict__ x, int ldx, const float *__restrict__ b, int K,
-              int Kp, int M, uint32_t *__restrict__ xp) {
+              int Kp, int M, int P, uint32_t *__restrict__ xp) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     const int64_t pairs_per_row = Kp / 2;
-    const int64_t total = 2 * static_cast<int64_t>(M) * pairs_per_row;
+    const int64_t total = static_cast<int64_t>(P) * M * pairs_per_row;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t pr = i % pairs_per_row;
@@ -358,9 +377,10 @@ size_t gemm_workspace_bytes(int N, int K, int P, int M) {
 }
 
 cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
-                        const float *b, int N, int K, const uint16_t *x, int M, int ldx,
+                        const float *b, int N, int K, int P, const uint16_t *x, int M, int ldx,
                         float *y, int ldy, void *workspace, uint32_t *fault_word,
                         uint64_t timeout_ns, int debug_flags) {
+    if (P != 2 && P != 3) return cudaErrorInvalidValue;
     const int Kp = static_cast<int>(padded_cols(K));
 
     cudaLaunchAttribute attr[1];
@@ -369,7 +389,7 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
 
     // 1. X'_k = fp16(x (.) b_k), permuted within 32-column groups.
     {
-        const int64_t total = 2 * static_cast<int64_t>(M) * (Kp / 2);
+        const int64_t total = static_cast<int64_t>(P) * M * (Kp / 2);
         int64_t blocks = (total + 255) / 256;
         if (blocks > static_cast<int64_t>(ctx.num_sms) * 16) blocks = static_cast<int64_t>(ctx.num_sms) * 16;
         cudaLaunchConfig_t cfg = {};
@@ -378,16 +398,16 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
         cfg.stream = ctx.stream;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, prep_x_kernel, x, ldx, b, K, Kp, M,
+        cudaError_t e = cudaLaunchKernelEx(&cfg, prep_x_kernel, x, ldx, b, K, Kp, M, P,
                                            static_cast<uint32_t *>(workspace));
         if (e != cudaSuccess) return e;
     }
 
-    // 2. Tensor map over the workspace viewed as [2][M][Kp] fp16.
+    // 2. Tensor map over the workspace viewed as [P][M][Kp] fp16.
     auto encode = get_encode_fn();
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap tmap;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), 2};
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(P)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kp) * 2, static_cast<cuuint64_t>(M) * Kp * 2};
     cuuint32_t box[3] = {kBK, kBN, 1};
     cuuint32_t estr[3] = {1, 1, 1};
@@ -413,13 +433,14 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     args.num_tiles = args.tiles_m * tiles_n;
     args.debug = debug_flags;
 
-    static int opted[64] = {};
+    void (*kern)(CUtensorMap, GemmArgs) = P == 2 ? gemm_kernel<2> : gemm_kernel<3>;
+    static int opted[2][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !opted[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (dev >= 0 && dev < 64 && !opted[P - 2][dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
-        opted[dev] = 1;
+        opted[P - 2][dev] = 1;
     }
     int grid = args.num_tiles < ctx.num_sms ? args.num_tiles : ctx.num_sms;
     cudaLaunchConfig_t cfg = {};
@@ -429,7 +450,7 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     cfg.stream = ctx.stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_kernel, tmap, args);
+    return cudaLaunchKernelEx(&cfg, kern, tmap, args);
 }
 
 }  // namespace rabit

@@ -32,6 +32,7 @@
 //    partials meet in shared memory.
 //  * RABIT_F32 activations use two 13-bit slices of a 24-bit z (twice the dp2a work).
 #include <algorithm>
+#include <type_traits>
 
 #include "rabit_device.cuh"
 #include "rabit_kernels.h"
@@ -40,6 +41,8 @@ namespace rabit {
 namespace {
 
 constexpr int kMaxThreads = 768;
+// fp32 activations (two slices per z value) and three paths need more registers per thread.
+__host__ __device__ constexpr int max_threads(bool f32x, int P) { return (f32x || P == 3) ? 512 : kMaxThreads; }
 constexpr int kGroupRows = 8;            // rows per butterfly reduction and per copy barrier
 constexpr int kSmemBudget = 200 * 1024;  // dynamic shared memory a CTA may use
 // A group's 16 z-pair words per path and slice sit together, 20 words apart from the next
@@ -48,9 +51,9 @@ constexpr int kSmemBudget = 200 * 1024;  // dynamic shared memory a CTA may use
 constexpr int kZStride = 20;
 
 struct GemvArgs {
-    const uint2 *packed;   // [N][Wr] groups {path-1 word, path-2 word}
-    const float *a;        // [2][N]
-    const float *b;        // [2][K]
+    const uint32_t *packed;  // [N][Wr] groups of G words: the paths' words (+ a zero word for 3)
+    const float *a;        // [P][N]
+    const float *b;        // [P][K]
     const void *x;         // [batch][ldx]
     float *y;              // [batch][ldy]
     uint32_t *fault;
@@ -60,29 +63,38 @@ struct GemvArgs {
     int pass_rows;         // rows staged in shared memory at a time (multiple of 8)
     int nchunks;           // 32-group chunks of a row
     int vec_x;             // x rows 16-byte aligned: 16-byte loads of 8 columns
-    int vec_b;             // both b rows 16-byte aligned
+    int vec_b;             // every b row 16-byte aligned
 };
+
+// Words per 32-column group: two paths as a uint2, three paths as a uint4 (the fourth word is
+// padding), as Appendix E.1 groups them.
+template <int kP> using GroupWords = typename std::conditional<kP == 2, uint2, uint4>::type;
+// Per-row output scales in shared memory: {a_1, a_2} or {a_1, a_2, a_3, 0}.
+template <int kP> using RowScales = typename std::conditional<kP == 2, float2, float4>::type;
 
 struct SmemLayout {
     uint32_t w, zp, zinit, zscale, arow, red, bar, total;
 };
 
 // Per-group tables have rows Wr + 1 words apart, which keeps their stores conflict-free.
-template <int kSlices>
+template <int kSlices, int kP>
 __host__ __device__ inline SmemLayout smem_layout(int pass_rows, int Wr, int nchunks) {
     SmemLayout L;
     uint32_t off = 0;
     auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 127u) & ~127u; return o; };
-    L.w = take(static_cast<uint32_t>(pass_rows) * Wr * 8u);
-    L.zp = take(static_cast<uint32_t>(kSlices) * 2u * Wr * kZStride * 4u);
-    L.zinit = take(static_cast<uint32_t>(kSlices) * 2u * (Wr + 1) * 4u);
-    L.zscale = take(2u * (Wr + 1) * 4u);
-    L.arow = take(static_cast<uint32_t>(pass_rows) * 8u);
+    L.w = take(static_cast<uint32_t>(pass_rows) * Wr * static_cast<uint32_t>(sizeof(GroupWords<kP>)));
+    L.zp = take(static_cast<uint32_t>(kSlices) * kP * Wr * kZStride * 4u);
+    L.zinit = take(static_cast<uint32_t>(kSlices) * kP * (Wr + 1) * 4u);
+    L.zscale = take(static_cast<uint32_t>(kP) * (Wr + 1) * 4u);
+    L.arow = take(static_cast<uint32_t>(pass_rows) * static_cast<uint32_t>(sizeof(RowScales<kP>)));
     L.red = take(static_cast<uint32_t>(nchunks) * pass_rows * 4u);
     L.bar = take(static_cast<uint32_t>(pass_rows / kGroupRows) * 8u);
     L.total = off;
     return L;
 }
+
+__device__ __forceinline__ uint32_t path_word(const uint2 &g, int k) { return k ? g.y : g.x; }
+__device__ __forceinline__ uint32_t path_word(const uint4 &g, int k) { return k == 0 ? g.x : (k == 1 ? g.y : g.z); }
 
 __device__ __forceinline__ uint32_t dp2a_lo(uint32_t zpair, uint32_t bytes, uint32_t acc) {
     uint32_t d;
@@ -116,11 +128,11 @@ __device__ __forceinline__ float load_x(const void *x, int64_t idx) {
     }
 }
 
-// Loads of one z task: 8 columns j0..j0+7 of x (batch row beta) and of both b rows.
+// Loads of one z task: 8 columns j0..j0+7 of x (batch row beta) and of every b row.
 // Columns at or past K read as 0 (the padding of the last group).
-template <bool kF32X>
+template <bool kF32X, int kP>
 __device__ __forceinline__ void load_ztask(const GemvArgs &p, int beta, int j0, bool on,
-                                           float (&xv)[8], float (&bv)[2][8]) {
+                                           float (&xv)[8], float (&bv)[kP][8]) {
     const int64_t xrow = static_cast<int64_t>(beta) * p.ldx;
     if (on && j0 + 8 <= p.K) {
         if (p.vec_x) {
@@ -144,7 +156,7 @@ __device__ __forceinline__ void load_ztask(const GemvArgs &p, int beta, int j0, 
             for (int i = 0; i < 8; ++i) xv[i] = load_x<kF32X>(p.x, xrow + j0 + i);
         }
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < kP; ++k) {
             const float *brow = p.b + static_cast<int64_t>(k) * p.K + j0;
             if (p.vec_b) {
                 const float4 u0 = __ldg(reinterpret_cast<const float4 *>(brow));
@@ -161,8 +173,8 @@ __device__ __forceinline__ void load_ztask(const GemvArgs &p, int beta, int j0, 
         for (int i = 0; i < 8; ++i) {
             const bool ok = on && j0 + i < p.K;
             xv[i] = ok ? load_x<kF32X>(p.x, xrow + j0 + i) : 0.0f;
-            bv[0][i] = ok ? __ldg(p.b + j0 + i) : 0.0f;
-            bv[1][i] = ok ? __ldg(p.b + p.K + j0 + i) : 0.0f;
+#pragma unroll
+            for (int k = 0; k < kP; ++k) bv[k][i] = ok ? __ldg(p.b + static_cast<int64_t>(k) * p.K + j0 + i) : 0.0f;
         }
     }
 }
@@ -190,17 +202,19 @@ __device__ __forceinline__ float butterfly8(const float (&v)[8], int lane) {
     return s;
 }
 
-template <bool kF32X>
-__global__ void __launch_bounds__(kMaxThreads, 1)
+template <bool kF32X, int kP>
+__global__ void __launch_bounds__(max_threads(kF32X, kP), 1)
 gemv_kernel(const GemvArgs p) {
     constexpr int kSlices = kF32X ? 2 : 1;
+    using WG = GroupWords<kP>;
+    using AS = RowScales<kP>;
     extern __shared__ __align__(128) uint8_t smem[];
-    const SmemLayout L = smem_layout<kSlices>(p.pass_rows, p.Wr, p.nchunks);
-    uint2 *wbuf = reinterpret_cast<uint2 *>(smem + L.w);             // [pass_rows][Wr]
+    const SmemLayout L = smem_layout<kSlices, kP>(p.pass_rows, p.Wr, p.nchunks);
+    WG *wbuf = reinterpret_cast<WG *>(smem + L.w);                   // [pass_rows][Wr]
     uint32_t *zp = reinterpret_cast<uint32_t *>(smem + L.zp);        // [slice][path][Wr][kZStride]
     int32_t *zinit = reinterpret_cast<int32_t *>(smem + L.zinit);    // [slice][path][zs]
     float *zscale = reinterpret_cast<float *>(smem + L.zscale);      // [path][zs]
-    float2 *arow = reinterpret_cast<float2 *>(smem + L.arow);        // [pass_rows]
+    AS *arow = reinterpret_cast<AS *>(smem + L.arow);                // [pass_rows]
     float *red = reinterpret_cast<float *>(smem + L.red);            // [nchunks][pass_rows]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar);     // [pass_rows / 8]
     const int zs = p.Wr + 1;
@@ -217,20 +231,17 @@ gemv_kernel(const GemvArgs p) {
         for (int g = 0; g < p.pass_rows / kGroupRows; ++g) mbar_init(smem_u32(&bars[g]), 1);
         fence_mbarrier_init();
         // L2 prefetch of this CTA's rows (one contiguous block)
-        const uint8_t *base = reinterpret_cast<const uint8_t *>(p.packed + static_cast<int64_t>(row_begin) * p.Wr);
-        const uint64_t bytes = static_cast<uint64_t>(row_end - row_begin) * p.Wr * 8u;
+        const uint8_t *base = reinterpret_cast<const uint8_t *>(
+            reinterpret_cast<const WG *>(p.packed) + static_cast<int64_t>(row_begin) * p.Wr);
+        const uint64_t bytes = static_cast<uint64_t>(row_end - row_begin) * p.Wr * sizeof(WG);
         for (uint64_t o = 0; o < bytes; o += (1u << 20))
             bulk_prefetch_l2(base + o, static_cast<uint32_t>(min(bytes - o, static_cast<uint64_t>(1u << 20))));
     } else if (warp == 1) {
-        for (int c = lane * 32; c < p.K; c += 32 * 32) {                 // 128-byte lines of b
-            prefetch_l2(p.b + c);
-            prefetch_l2(p.b + p.K + c);
-        }
+        for (int c = lane * 32; c < p.K; c += 32 * 32)                   // 128-byte lines of b
+            for (int k = 0; k < kP; ++k) prefetch_l2(p.b + static_cast<int64_t>(k) * p.K + c);
     } else if (warp == 2) {
-        for (int r = lane * 32; r < row_end - row_begin; r += 32 * 32) { // lines of a
-            prefetch_l2(p.a + row_begin + r);
-            prefetch_l2(p.a + p.N + row_begin + r);
-        }
+        for (int r = lane * 32; r < row_end - row_begin; r += 32 * 32)   // lines of a
+            for (int k = 0; k < kP; ++k) prefetch_l2(p.a + static_cast<int64_t>(k) * p.N + row_begin + r);
     } else if (warp == 3) {
         const int per_line = kF32X ? 32 : 64;
         for (int beta = 0; beta < p.batch; ++beta)
@@ -250,11 +261,12 @@ gemv_kernel(const GemvArgs p) {
         if (warp == 0) {
             for (int g = lane; g < ngroups; g += 32) {
                 const int rows_g = min(kGroupRows, prows - g * kGroupRows);
-                const uint32_t bytes = static_cast<uint32_t>(rows_g) * p.Wr * 8u;
+                const uint32_t bytes = static_cast<uint32_t>(rows_g) * p.Wr * static_cast<uint32_t>(sizeof(WG));
                 const uint32_t bar = smem_u32(&bars[g]);
                 mbar_arrive_expect_tx(bar, bytes);
                 bulk_g2s(smem_u32(wbuf + static_cast<int64_t>(g) * kGroupRows * p.Wr),
-                         p.packed + static_cast<int64_t>(pr0 + g * kGroupRows) * p.Wr, bytes, bar);
+                         reinterpret_cast<const WG *>(p.packed) + static_cast<int64_t>(pr0 + g * kGroupRows) * p.Wr,
+                         bytes, bar);
             }
         }
         for (int beta = 0; beta < p.batch; ++beta) {
@@ -262,17 +274,24 @@ gemv_kernel(const GemvArgs p) {
             // 4 consecutive threads per group, 8 columns each; x is read once for both paths.
             // The loads of kZBatch tasks are issued before any of them is used, and a's values
             // for the pass are fetched alongside, so the stage waits on memory about once.
-            float2 apre = make_float2(0.0f, 0.0f);
-            if (beta == 0 && tid < prows) apre = make_float2(__ldg(p.a + pr0 + tid), __ldg(p.a + p.N + pr0 + tid));
+            auto load_scales = [&](int r) -> AS {
+                if constexpr (kP == 2)
+                    return make_float2(__ldg(p.a + pr0 + r), __ldg(p.a + p.N + pr0 + r));
+                else
+                    return make_float4(__ldg(p.a + pr0 + r), __ldg(p.a + p.N + pr0 + r),
+                                       __ldg(p.a + 2 * static_cast<int64_t>(p.N) + pr0 + r), 0.0f);
+            };
+            AS apre{};
+            if (beta == 0 && tid < prows) apre = load_scales(tid);
             constexpr int kZBatch = 2;
             const int ztasks = 4 * p.Wr;
             const int ztasks_pad = (ztasks + 31) & ~31;
             for (int t0 = tid; t0 < ztasks_pad; t0 += kZBatch * nthreads) {
-                float xv[kZBatch][8], zv[kZBatch][2][8];
+                float xv[kZBatch][8], zv[kZBatch][kP][8];
 #pragma unroll
                 for (int u = 0; u < kZBatch; ++u) {
                     const int t = t0 + u * nthreads;
-                    load_ztask<kF32X>(p, beta, (t >> 2) * 32 + 8 * (t & 3), t < ztasks, xv[u], zv[u]);
+                    load_ztask<kF32X, kP>(p, beta, (t >> 2) * 32 + 8 * (t & 3), t < ztasks, xv[u], zv[u]);
                 }
 #pragma unroll
                 for (int u = 0; u < kZBatch; ++u) {
@@ -283,7 +302,7 @@ gemv_kernel(const GemvArgs p) {
                     const int gloc = on ? (t >> 2) : 0;
                     const int h = q >> 1, half = q & 1;  // columns 8q..8q+7 of the group
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
+                    for (int k = 0; k < kP; ++k) {
                         float m = 0.0f;
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -323,7 +342,7 @@ gemv_kernel(const GemvArgs p) {
                                 if (on) {
                                     const int zpre = part[s] << (3 - qb);      // weight 2^(3-q)
                                     uint16_t *slot = reinterpret_cast<uint16_t *>(
-                                        zp + ((s * 2 + k) * p.Wr + gloc) * kZStride + pair) + half;
+                                        zp + ((s * kP + k) * p.Wr + gloc) * kZStride + pair) + half;
                                     *slot = static_cast<uint16_t>(zpre & 0xFFFF);
                                 }
                             }
@@ -335,7 +354,7 @@ gemv_kernel(const GemvArgs p) {
                         }
                         if (on && q == 0) {
 #pragma unroll
-                            for (int s = 0; s < kSlices; ++s) zinit[(s * 2 + k) * zs + gloc] = -4 * zsum[s];
+                            for (int s = 0; s < kSlices; ++s) zinit[(s * kP + k) * zs + gloc] = -4 * zsum[s];
                             // the accumulator ends at -4T and t = T * 2^-e
                             zscale[k * zs + gloc] = -__uint_as_float(static_cast<uint32_t>(125 - e) << 23);
                         }
@@ -345,9 +364,8 @@ gemv_kernel(const GemvArgs p) {
             if (beta == 0) {
                 if (tid < prows) arow[tid] = apre;
                 for (int r = tid + nthreads; r < p.pass_rows; r += nthreads)   // rows past prows: a = 0
-                    arow[r] = r < prows ? make_float2(__ldg(p.a + pr0 + r), __ldg(p.a + p.N + pr0 + r))
-                                        : make_float2(0.0f, 0.0f);
-                if (tid >= prows && tid < p.pass_rows) arow[tid] = make_float2(0.0f, 0.0f);
+                    arow[r] = r < prows ? load_scales(r) : AS{};
+                if (tid >= prows && tid < p.pass_rows) arow[tid] = AS{};
             }
             __syncthreads();
 
@@ -362,28 +380,27 @@ gemv_kernel(const GemvArgs p) {
                 const int gl = c * 32 + lane;
                 const bool lane_on = gl < p.Wr;
                 const int gz = lane_on ? gl : p.Wr - 1;     // lanes past the row read a valid word
-                float sk[2];
-                if (beta == 0 && !mbar_wait_bounded(smem_u32(&bars[g]), parity, &abort_flag,
-                                                    p.timeout_ns, p.fault, FAULT_GEMV_WAIT_COPY))
-                    sk[0] = sk[1] = 0.0f;  // the copy never landed: contribute nothing
-                else
+                float sk[kP];
+                const bool landed = beta != 0 || mbar_wait_bounded(smem_u32(&bars[g]), parity, &abort_flag,
+                                                                   p.timeout_ns, p.fault, FAULT_GEMV_WAIT_COPY);
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) sk[k] = lane_on ? zscale[k * zs + gz] : 0.0f;
-                uint2 w[kGroupRows];
-                const uint2 *wrow = wbuf + static_cast<int64_t>(g) * kGroupRows * p.Wr + gz;
+                for (int k = 0; k < kP; ++k)   // a copy that never landed contributes nothing
+                    sk[k] = landed && lane_on ? zscale[k * zs + gz] : 0.0f;
+                WG w[kGroupRows];
+                const WG *wrow = wbuf + static_cast<int64_t>(g) * kGroupRows * p.Wr + gz;
 #pragma unroll
                 for (int i = 0; i < kGroupRows; ++i) w[i] = wrow[static_cast<int64_t>(i) * p.Wr];
-                float tk[2][kGroupRows];
+                float tk[kP][kGroupRows];
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
+                for (int k = 0; k < kP; ++k) {
                     int32_t acc[kSlices][kGroupRows];
                     uint4 zq[kSlices][4];
 #pragma unroll
                     for (int s = 0; s < kSlices; ++s) {
-                        const uint4 *zrow = reinterpret_cast<const uint4 *>(zp + ((s * 2 + k) * p.Wr + gz) * kZStride);
+                        const uint4 *zrow = reinterpret_cast<const uint4 *>(zp + ((s * kP + k) * p.Wr + gz) * kZStride);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) zq[s][j] = zrow[j];
-                        const int32_t init = zinit[(s * 2 + k) * zs + gz];
+                        const int32_t init = zinit[(s * kP + k) * zs + gz];
 #pragma unroll
                         for (int i = 0; i < kGroupRows; ++i) acc[s][i] = init;
                     }
@@ -393,7 +410,7 @@ gemv_kernel(const GemvArgs p) {
                     for (int s4 = 0; s4 < 2; ++s4) {
 #pragma unroll
                         for (int i = 0; i < kGroupRows; ++i) {
-                            const uint32_t wv = (k ? w[i].y : w[i].x) >> (4 * s4);
+                            const uint32_t wv = path_word(w[i], k) >> (4 * s4);
 #pragma unroll
                             for (int s = 0; s < kSlices; ++s) {
                                 uint32_t a0 = static_cast<uint32_t>(acc[s][i]);
@@ -417,12 +434,20 @@ gemv_kernel(const GemvArgs p) {
                     }
                 }
                 float part[kGroupRows];
-                const float4 *a4 = reinterpret_cast<const float4 *>(arow + g * kGroupRows);
+                if constexpr (kP == 2) {
+                    const float4 *a4 = reinterpret_cast<const float4 *>(arow + g * kGroupRows);
 #pragma unroll
-                for (int i = 0; i < kGroupRows / 2; ++i) {
-                    const float4 av = a4[i];
-                    part[2 * i] = fmaf(av.x, tk[0][2 * i], av.y * tk[1][2 * i]);
-                    part[2 * i + 1] = fmaf(av.z, tk[0][2 * i + 1], av.w * tk[1][2 * i + 1]);
+                    for (int i = 0; i < kGroupRows / 2; ++i) {
+                        const float4 av = a4[i];
+                        part[2 * i] = fmaf(av.x, tk[0][2 * i], av.y * tk[1][2 * i]);
+                        part[2 * i + 1] = fmaf(av.z, tk[0][2 * i + 1], av.w * tk[1][2 * i + 1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kGroupRows; ++i) {
+                        const float4 av = arow[g * kGroupRows + i];
+                        part[i] = fmaf(av.x, tk[0][i], fmaf(av.y, tk[1][i], av.z * tk[2][i]));
+                    }
                 }
                 const float total = butterfly8(part, lane);
                 const int ri = g * kGroupRows + ((lane >> 2) & 7);
@@ -448,32 +473,34 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 }  // namespace
 
 cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
-                        const float *b, int N, int K, const void *x, bool x_bf16, int batch,
+                        const float *b, int N, int K, int P, const void *x, bool x_bf16, int batch,
                         int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns) {
+    if (P != 2 && P != 3) return cudaErrorInvalidValue;
     const int Wr = static_cast<int>(padded_cols(K) / 32);
     const int nchunks = ceil_div(Wr, 32);
     // Rows: as evenly as possible over the SMs, one CTA each.
     const int rows_per_cta = ceil_div(N, std::min(ctx.num_sms, N));
     const int grid = ceil_div(N, rows_per_cta);
     const bool f32x = !x_bf16;
-    auto bytes_for = [&](int rows) {
-        return f32x ? smem_layout<2>(rows, Wr, nchunks).total : smem_layout<1>(rows, Wr, nchunks).total;
+    auto bytes_for = [&](int rows) -> uint32_t {
+        if (P == 2) return f32x ? smem_layout<2, 2>(rows, Wr, nchunks).total : smem_layout<1, 2>(rows, Wr, nchunks).total;
+        return f32x ? smem_layout<2, 3>(rows, Wr, nchunks).total : smem_layout<1, 3>(rows, Wr, nchunks).total;
     };
     int pass_rows = ceil_div(rows_per_cta, kGroupRows) * kGroupRows;
     while (pass_rows > kGroupRows && bytes_for(pass_rows) > static_cast<uint32_t>(kSmemBudget))
         pass_rows -= kGroupRows;
     if (bytes_for(pass_rows) > static_cast<uint32_t>(kSmemBudget)) return cudaErrorInvalidConfiguration;
     // Warps: as few as give every warp the same number of work items (8 rows x 32 groups)
-    // within kMaxThreads, but enough that the z stage has at most two tasks per thread
+    // within the thread budget, but enough that the z stage has at most two tasks per thread
     // (up to 16 warps).
     const int items = ceil_div(pass_rows, kGroupRows) * nchunks;
-    const int max_warps = kMaxThreads / 32;
+    const int max_warps = max_threads(f32x, P) / 32;
     const int per_warp = ceil_div(items, max_warps);
     const int zwarps = std::min(16, ceil_div(4 * Wr, 64));
     const int threads = 32 * std::min(max_warps, std::max(ceil_div(items, per_warp), zwarps));
 
     GemvArgs p;
-    p.packed = reinterpret_cast<const uint2 *>(packed);
+    p.packed = packed;
     p.a = a;
     p.b = b;
     p.x = x;
@@ -494,15 +521,17 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     p.vec_b = (reinterpret_cast<uintptr_t>(b) % 16 == 0) && (K % 4 == 0);
 
     const uint32_t smem = bytes_for(pass_rows);
-    auto kern = f32x ? gemv_kernel<true> : gemv_kernel<false>;
+    void (*kern)(GemvArgs) = P == 2 ? (f32x ? gemv_kernel<true, 2> : gemv_kernel<false, 2>)
+                                    : (f32x ? gemv_kernel<true, 3> : gemv_kernel<false, 3>);
+    const int variant = (P == 3 ? 2 : 0) + (f32x ? 1 : 0);
     // Opt in to the largest dynamic shared memory once per kernel and device.
-    static int opted[2][64] = {};
+    static int opted[4][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !opted[f32x][dev]) {
+    if (dev >= 0 && dev < 64 && !opted[variant][dev]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
         if (e != cudaSuccess) return e;
-        opted[f32x][dev] = 1;
+        opted[variant][dev] = 1;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));

@@ -105,12 +105,12 @@ int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ldw, int P, 
     if (w_dtype != RABIT_F32 && w_dtype != RABIT_BF16) return RABIT_ERR_INVALID_ARG;
     if (!W || !a || !b || !packed) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || P < 1 || ldw < K) return RABIT_ERR_SHAPE;
-    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
     if (!aligned(packed, 16)) return RABIT_ERR_ALIGNMENT;
     rabit::LaunchCtx ctx;
     int st = device_ctx(stream, ctx, nullptr);
     if (st != RABIT_OK) return st;
-    return finish_launch(rabit::launch_derive_pack(ctx, W, w_dtype == RABIT_BF16, N, K, ldw, a, b, packed));
+    return finish_launch(rabit::launch_derive_pack(ctx, W, w_dtype == RABIT_BF16, N, K, ldw, P, a, b, packed));
 }
 
 int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
@@ -119,14 +119,14 @@ int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, in
     if (!packed || !a || !b || !x || !y) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || P < 1 || batch < 1 || batch > 16 || ldx < K || ldy < N)
         return RABIT_ERR_SHAPE;
-    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
     if (!aligned(packed, 16)) return RABIT_ERR_ALIGNMENT;
     if (!aligned(x, x_dtype == RABIT_BF16 ? 2 : 4) || !aligned(y, 4)) return RABIT_ERR_ALIGNMENT;
     rabit::LaunchCtx ctx;
     uint32_t *fault = nullptr;
     int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
-    return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, x, x_dtype == RABIT_BF16,
+    return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, P, x, x_dtype == RABIT_BF16,
                                             batch, ldx, y, ldy, fault, wait_timeout_ns()));
 }
 
@@ -135,7 +135,7 @@ int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, in
                size_t workspace_bytes, void *stream) {
     if (!packed || !a || !b || !x_bf16 || !y) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || P < 1 || M < 1 || ldx < K || ldy < N) return RABIT_ERR_SHAPE;
-    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
     if (!aligned(packed, 16) || !aligned(x_bf16, 16) || (ldx % 8) != 0 || !aligned(y, 4))
         return RABIT_ERR_ALIGNMENT;
     if (!workspace || workspace_bytes < rabit::gemm_workspace_bytes(N, K, P, M))
@@ -147,7 +147,7 @@ int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, in
     if (st != RABIT_OK) return st;
     const uint64_t timeout_ns = wait_timeout_ns();
     const int debug = env_flag("RABIT_TEST_SKIP_ONE_ARRIVE") ? 1 : 0;
-    return finish_launch(rabit::launch_gemm(ctx, packed, a, b, N, K, x_bf16, M, ldx, y, ldy,
+    return finish_launch(rabit::launch_gemm(ctx, packed, a, b, N, K, P, x_bf16, M, ldx, y, ldy,
                                             workspace, fault, timeout_ns, debug));
 }
 
@@ -157,7 +157,7 @@ int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, i
                        const uint16_t *x_bf16, int M, int ldx, float *y, int ldy, void *stream) {
     if (!packed || !a || !b || !x_bf16 || !y) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || P < 1 || M < 1 || ldx < K || ldy < N) return RABIT_ERR_SHAPE;
-    if (P != 2) return RABIT_ERR_UNSUPPORTED;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
     if (!aligned(packed, 16) || !aligned(x_bf16, 16) || (ldx % 8) != 0 || !aligned(y, 4))
         return RABIT_ERR_ALIGNMENT;
     const size_t need = rabit::gemm_workspace_bytes(N, K, P, M);
@@ -173,7 +173,7 @@ int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, i
     if (need > scratch_bytes) return RABIT_ERR_WORKSPACE;
     const uint64_t timeout_ns = wait_timeout_ns();
     const int debug = env_flag("RABIT_TEST_SKIP_ONE_ARRIVE") ? 1 : 0;
-    return finish_launch(rabit::launch_gemm(ctx, packed, a, b, N, K, x_bf16, M, ldx, y, ldy,
+    return finish_launch(rabit::launch_gemm(ctx, packed, a, b, N, K, P, x_bf16, M, ldx, y, ldy,
                                             scratch, fault, timeout_ns, debug));
 }
 

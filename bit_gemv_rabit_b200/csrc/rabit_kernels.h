@@ -18,18 +18,19 @@ struct LaunchCtx {
     bool pdl;
 };
 
+// P = 2 or 3 paths.
 cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16, int N, int K,
-                               int ldw, const float *a, const float *b, uint32_t *packed);
+                               int ldw, int P, const float *a, const float *b, uint32_t *packed);
 
 cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
-                        const float *b, int N, int K, const void *x, bool x_bf16, int batch,
+                        const float *b, int N, int K, int P, const void *x, bool x_bf16, int batch,
                         int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
 // Device address and size of the library's fixed GEMM scratch buffer (rabit_gemm_noalloc).
 cudaError_t gemm_noalloc_scratch(void **ptr, size_t *bytes);
 cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
-                        const float *b, int N, int K, const uint16_t *x, int M, int ldx,
+                        const float *b, int N, int K, int P, const uint16_t *x, int M, int ldx,
                         float *y, int ldy, void *workspace, uint32_t *fault_word,
                         uint64_t timeout_ns, int debug_flags);
 

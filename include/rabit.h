@@ -53,7 +53,7 @@ typedef enum rabit_status {
     RABIT_ERR_INVALID_ARG = -1,  /* null pointer, bad enum value */
     RABIT_ERR_ALIGNMENT = -2,    /* a pointer or pitch breaks the stated alignment */
     RABIT_ERR_SHAPE = -3,        /* N, K, M, batch or a pitch out of range */
-    RABIT_ERR_UNSUPPORTED = -4,  /* valid request this build does not implement (P != 2) */
+    RABIT_ERR_UNSUPPORTED = -4,  /* valid request this build does not implement (P other than 2, 3) */
     RABIT_ERR_WORKSPACE = -5,    /* workspace missing or too small */
     RABIT_ERR_ARCH = -6,         /* current device is not sm_100 */
     RABIT_ERR_CUDA = -7,         /* a CUDA runtime call failed; see rabit_last_cuda_error() */
@@ -62,13 +62,15 @@ typedef enum rabit_status {
 
 /*
  * Packed sign layout RABIT_LAYOUT_V2 (Appendix E.1 "Weight Packing": 32 columns per
- * uint32 word, +1 -> bit 0, -1 -> bit 1, the 2-bit case's two words grouped as a uint2).
- *   Kp = ceil(K/128)*128, Wr = Kp/32 groups of 32 columns per row;
+ * uint32 word, +1 -> bit 0, -1 -> bit 1, the 2-bit case's two words grouped as a uint2 and
+ * the 3-bit case's three words plus one padding word as a uint4).
+ *   Kp = ceil(K/128)*128, Wr = Kp/32 groups of 32 columns per row, G = 2 (P = 2) or 4 (P = 3);
  *   column j sits at bit (j % 32) of group j/32, least significant bit first;
- *   word(k, n, w) = (n*Wr + w)*2 + k    (path k in {0,1}, row n < N, group w < Wr).
- * Rows are stored one after another (row pitch Kp/4 bytes), and inside a row the two
- * paths' words of each 32-column group sit side by side.  Padding columns (j >= K) are 0;
- * rows are not padded.  The buffer holds 2*N*Wr uint32 words and must be 16-byte aligned.
+ *   word(k, n, w) = (n*Wr + w)*G + k    (path k < P, row n < N, group w < Wr).
+ * Rows are stored one after another, and inside a row the paths' words of each 32-column
+ * group sit side by side.  Padding columns (j >= K) and the padding word of a 3-path group
+ * are 0; rows are not padded.  The buffer holds G*N*Wr uint32 words (rabit_packed_words)
+ * and must be 16-byte aligned.
  */
 #define RABIT_LAYOUT_V2 2
 RABIT_API size_t rabit_packed_words(int N, int K, int P);
@@ -77,14 +79,18 @@ RABIT_API size_t rabit_packed_words(int N, int K, int P);
  * rabit_derive_pack -- sec. 4.2 "The Coupled Forward Pass", steps 1-3, followed by the
  * Appendix E.1 packing.  For every n < N, j < K:
  *     s1 = sign(W[n][j]);  r1 = W[n][j] - a[0][n]*s1*b[0][j];  s2 = sign(r1)
- * r1 is formed with one rounding (fused multiply-add), so its sign is exact whenever the
- * exact residual is nonzero and |a[0][n]*b[0][j]| >= 2^-100.  Writes every word of the
- * packed buffer, padding columns included (so it never needs clearing).  Scales are read, never
- * written: they stay caller-owned learnable parameters.
+ * and for P = 3 the same rule once more (sec. 4.1 stacking):
+ *     r2 = r1 - a[1][n]*s2*b[1][j];  s3 = sign(r2)
+ * sign(v) = +1 unless v < 0.  With P = 2, r1 is formed with one rounding (fused
+ * multiply-add), so its sign is exact whenever the exact residual is nonzero and
+ * |a[0][n]*b[0][j]| >= 2^-100.  With P = 3 both residuals are formed in binary64 (each
+ * product exact, each subtraction rounded once).  Writes every word of the packed buffer,
+ * padding included (so it never needs clearing).  Scales are read, never written: they stay
+ * caller-owned learnable parameters.
  *   W       [N][ldw] fp32 (w_dtype RABIT_F32) or bf16 (RABIT_BF16), ldw >= K
- *   a       [P][N] fp32, b [P][K] fp32 (only path 1 is read when P = 2)
+ *   a       [P][N] fp32, b [P][K] fp32 (paths 1..P-1 are read; the last path needs no scale)
  *   packed  rabit_packed_words(N, K, P) uint32, 16-byte aligned (output)
- * Errors: INVALID_ARG (null, bad dtype), SHAPE (N, K < 1, ldw < K), UNSUPPORTED (P != 2),
+ * Errors: INVALID_ARG (null, bad dtype), SHAPE (N, K < 1, ldw < K), UNSUPPORTED (P not 2 or 3),
  *         ALIGNMENT (packed), ARCH, CUDA.
  */
 RABIT_API int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ldw, int P,

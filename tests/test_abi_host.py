@@ -45,9 +45,12 @@ def test_every_declared_symbol_is_exported(lib):
 def test_packed_words_matches_layout_definition(lib):
     for N, K in [(1, 1), (32, 128), (33, 129), (4096, 4096), (11008, 4096), (4096, 14336)]:
         assert lib.rabit_packed_words(N, K, 2) == oracle.packed_words(N, K, 2)
+    for N, K in [(1, 1), (33, 129), (4096, 4096)]:
+        assert lib.rabit_packed_words(N, K, 3) == oracle.packed_words(N, K, 3)
     assert lib.rabit_packed_words(0, 5, 2) == 0
     assert lib.rabit_gemm_workspace_bytes(4096, 4096, 2, 2048) == 2 * 2048 * 4096 * 2
     assert lib.rabit_gemm_workspace_bytes(10, 200, 2, 3) == 2 * 3 * 256 * 2
+    assert lib.rabit_gemm_workspace_bytes(10, 200, 3, 3) == 3 * 3 * 256 * 2
 
 
 def test_status_strings(lib):
@@ -63,7 +66,7 @@ def test_derive_pack_validation(lib):
     assert f(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), None, None) == INVALID      # null out
     assert f(P(FAKE), 0, 0, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None) == SHAPE     # N = 0
     assert f(P(FAKE), 0, 4, 4, 3, 2, P(FAKE), P(FAKE), P(FAKE), None) == SHAPE     # ldw < K
-    assert f(P(FAKE), 0, 4, 4, 4, 3, P(FAKE), P(FAKE), P(FAKE), None) == UNSUP     # P = 3
+    assert f(P(FAKE), 0, 4, 4, 4, 4, P(FAKE), P(FAKE), P(FAKE), None) == UNSUP     # P = 4
     assert f(P(FAKE), 0, 4, 4, 4, 1, P(FAKE), P(FAKE), P(FAKE), None) == UNSUP     # P = 1
     assert f(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE + 4), None) == ALIGN
 
@@ -81,7 +84,7 @@ def test_gemv_validation(lib):
     assert f(*args(ldx=7)) == SHAPE
     assert f(*args(ldy=7)) == SHAPE
     assert f(*args(K=0)) == SHAPE
-    assert f(*args(P=3)) == UNSUP
+    assert f(*args(P=4)) == UNSUP
     assert f(*args(packed=FAKE + 8)) == ALIGN
     assert f(*args(x=FAKE + 1)) == ALIGN
     assert f(*args(y=FAKE + 2)) == ALIGN
