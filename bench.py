@@ -200,16 +200,16 @@ def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
     return t.to(device)
 
 
-def make_layer(rabit, spec, idx, name, N, K, device, batch):
+def make_layer(rabit, spec, idx, name, N, K, device, batch, P=2):
     seed = inputs.seed_for(spec["cfg"], idx)
     W = inputs.weight(seed, N, K, sigma=spec["sigma"], outlier_frac=spec["w_outliers"])
-    a, b = inputs.scales(seed, W)
+    a, b = inputs.scales(seed, W, P=P)
     at = torch.from_numpy(a).to(device)
     bt = torch.from_numpy(b).to(device)
-    packed = rabit.alloc_packed(N, K, device=device)
-    rabit.rabit_derive_pack(torch.from_numpy(W).to(device), at, bt, packed)
+    packed = rabit.alloc_packed(N, K, P=P, device=device)
+    rabit.rabit_derive_pack(torch.from_numpy(W).to(device), at, bt, packed, P=P)
     x = inputs.activations(seed, batch, K, channel_outlier_frac=spec["x_outliers"])
-    return dict(name=name, N=N, K=K, a=at, b=bt, packed=packed, x_host=x,
+    return dict(name=name, N=N, K=K, P=P, a=at, b=bt, packed=packed, x_host=x,
                 x=bf16_tensor(x, device), y=torch.empty((batch, N), device=device))
 
 
@@ -303,6 +303,51 @@ def bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained):
                          "unit": "TFLOP/s", "frac": round(tflops / tf_peak, 4),
                          "peak_note": "measured dense bf16 burst; fp16 operands have the same nominal rate",
                          "frac_of_nominal_fp8_dense_4500": round(tflops / 4500.0, 4)}}
+
+
+def warm_launch_us(rabit, layers, device):
+    """Microseconds per launch of each distinct shape, re-reading the same weights 200 times
+    in a graph (L2-resident after the first launch: the warm-cache setting of the pages'
+    kernel-latency table)."""
+    out = {}
+    for L in layers:
+        key = f"{L['N']}x{L['K']}"
+        if key in out:
+            continue
+        g = capture_graph(lambda L=L: [rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"],
+                                                        L["x"], L["y"], P=L["P"]) for _ in range(200)])
+        out[key] = round(timed_replays([g], 5, 2, None, device) / 5 / 200 * 1e3, 2)
+    return out
+
+
+def bench_gemv_three_path(rabit, device, alu_peak):
+    """The 3-bit variant (three paths) on the same Llama-2-7B decode set, batch 1, ten rotated
+    copies (the pages' Table 7 reports 3-bit kernel latencies beside the 2-bit ones)."""
+    spec = inputs.WORKLOADS[WORKLOAD]
+    base = [make_layer(rabit, spec, idx, name, N, K, device, 1, P=3)
+            for idx, (name, N, K) in enumerate(spec["set"])]
+    sets = [base] + [[dict(L, packed=L["packed"].clone()) for L in base] for _ in range(COPIES - 1)]
+    torch.cuda.synchronize()
+
+    def step_fn(layers):
+        def f():
+            for L in layers:
+                rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"], P=3)
+        return f
+
+    graphs = [capture_graph(step_fn(ls)) for ls in sets]
+    steps = 2000
+    ms = timed_replays(graphs, steps, 50, None, device)
+    sign = sum(3 * L["N"] * (((L["K"] + 127) // 128) * 128) // 8 for L in base)
+    algo = sum(3 * L["N"] * (((L["K"] + 127) // 128) * 128) // 8 + 4 * 3 * (L["N"] + L["K"])
+               + L["K"] * 2 + L["N"] * 4 for L in base)
+    return {"workload": "llama2_7b_decode_b1_3path", "value": round(algo * steps / (ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "us_per_set": round(ms / steps * 1e3, 2),
+            "us_per_launch_warm_l2_by_shape": warm_launch_us(rabit, base, device),
+            "roofline": {"bound": "alu", "achieved": round(sign * steps / (ms * 1e-3) / 1e9, 1),
+                         "peak": round(alu_peak, 1), "unit": "GB/s",
+                         "frac": round(sign * steps / (ms * 1e-3) / 1e9 / alu_peak, 4)},
+            "note": "3 sign words + 1 padding word per group in HBM; algorithmic bytes count the 3 signs"}
 
 
 def bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained):
@@ -538,6 +583,8 @@ def run_ours(args, rank, world, local, dist):
     }
     if clocks is not None:
         line["clocks"] = clocks.summary()
+    if rank == 0 and world == 1 and not args.no_secondary:
+        line["us_per_launch_warm_l2_by_shape"] = warm_launch_us(rabit, base, device)
     traffic = _load_traffic()
     if traffic is not None:
         line["roofline"]["traffic"] = traffic
@@ -548,6 +595,8 @@ def run_ours(args, rank, world, local, dist):
         line["gemm"] = bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained)
         torch.cuda.empty_cache()
         line.update(bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained))
+        torch.cuda.empty_cache()
+        line["gemv_3path"] = bench_gemv_three_path(rabit, device, alu_peak)
         torch.cuda.empty_cache()
         prepare_oracle_inputs(base, spec)
         line["cpu_baseline"] = cpu_baseline(base, 1)
