@@ -57,6 +57,8 @@ def _load():
         lib.oracle_unpack.restype = None
         lib.oracle_layer.argtypes = [p, i64, p, i64, i64, ctypes.c_int, p, p, p, i64, i64, p]
         lib.oracle_layer.restype = None
+        lib.oracle_scale_grads.argtypes = [p, i64, i64, p, ctypes.c_int, p, p, p, p]
+        lib.oracle_scale_grads.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -155,3 +157,18 @@ def layer(S: np.ndarray, a: np.ndarray, b: np.ndarray, x: np.ndarray,
     _load().oracle_layer(_ptr(S), R, None if rows_arr is None else _ptr(rows_arr), N, K, P,
                          _ptr(ad), _ptr(bd), _ptr(xd), B, K, _ptr(y))
     return y
+
+
+def scale_grads(G: np.ndarray, S: np.ndarray, a: np.ndarray, b: np.ndarray):
+    """Scale gradients for G = dL/dW_hat with the signs held fixed (chain rule on sec. 4.1's
+    W_hat = sum_k a_k S_k b_k): ga[k][n] = sum_j G S_k b_k, gb[k][j] = sum_n G a_k S_k.
+    Returns float64 (ga [P][N], gb [P][K])."""
+    S = np.ascontiguousarray(S, dtype=np.int8)
+    P, N, K = S.shape
+    Gd = np.ascontiguousarray(widen(G)).reshape(N, K)
+    ad = np.ascontiguousarray(widen(a)).reshape(-1, N)
+    bd = np.ascontiguousarray(widen(b)).reshape(-1, K)
+    ga = np.empty((P, N), dtype=np.float64)
+    gb = np.empty((P, K), dtype=np.float64)
+    _load().oracle_scale_grads(_ptr(Gd), N, K, _ptr(S), P, _ptr(ad), _ptr(bd), _ptr(ga), _ptr(gb))
+    return ga, gb

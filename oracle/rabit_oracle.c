@@ -151,6 +151,38 @@ ORACLE_API void oracle_layer(const int8_t *S, int64_t R, const int64_t *rows, in
     }
 }
 
+/*
+ * Gradients of the layer's scales for a given gradient G = dL/dW_hat (the straight-through
+ * estimator passes G to the shared weight unchanged and holds the signs fixed; the pages'
+ * sec. 4.2 update formula is lost in extraction, so this is the plain chain rule applied to
+ * sec. 4.1's W_hat = sum_k a_k (.) S_k (.) b_k):
+ *   ga[k][n] = sum_j G[n][j] * S_k[n][j] * b_k[j]
+ *   gb[k][j] = sum_n G[n][j] * a_k[n] * S_k[n][j]
+ *   G  : float64 [N][K];  S : int8 [P][N][K];  a : [P][N];  b : [P][K]
+ *   ga : float64 [P][N];  gb : float64 [P][K]
+ */
+ORACLE_API void oracle_scale_grads(const double *G, int64_t N, int64_t K, const int8_t *S, int P,
+                                   const double *a, const double *b, double *ga, double *gb)
+{
+    for (int k = 0; k < P; ++k) {
+        const int8_t *Sk = S + (int64_t)k * N * K;
+        #pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            double t = 0.0;
+            for (int64_t j = 0; j < K; ++j)
+                t += G[n * K + j] * (double)Sk[n * K + j] * b[(int64_t)k * K + j];
+            ga[(int64_t)k * N + n] = t;
+        }
+        #pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < K; ++j) {
+            double t = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                t += G[n * K + j] * a[(int64_t)k * N + n] * (double)Sk[n * K + j];
+            gb[(int64_t)k * K + j] = t;
+        }
+    }
+}
+
 /* Number of OpenMP threads the parallel loops above use (1 without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

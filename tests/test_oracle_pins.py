@@ -371,3 +371,37 @@ def test_three_path_layer_matches_numpy_matmul():
     x = inputs.bf16_to_f32(inputs.activations(74, 3, 130)).astype(np.float64)
     W_hat = sum(np.outer(a[k].astype(np.float64), b[k].astype(np.float64)) * S[k] for k in range(3))
     np.testing.assert_allclose(oracle.layer(S, a, b, x), x @ W_hat.T, rtol=1e-12, atol=1e-14)
+
+
+# ---- scale gradients (the layer's backward for a and b with the signs held fixed)
+
+def test_scale_grads_match_finite_differences_of_the_layer():
+    # L(a, b) = sum_{m,n} dY[m][n] * y[m][n] is linear in each a_k[n] and each b_k[j], so a
+    # difference quotient of the pinned layer is exact up to float64 rounding.
+    N, K, M = 12, 70, 5
+    W, a, b = _three_path_layer(91, N, K)
+    S = oracle.derive_signs(W, a, b, P=3)
+    rng = np.random.default_rng(91)
+    x = rng.standard_normal((M, K))
+    dY = rng.standard_normal((M, N))
+    G = dY.T @ x                                             # dL/dW_hat for y = x W_hat^T
+    ga, gb = oracle.scale_grads(G, S, a, b)
+    ad, bd = a.astype(np.float64), b.astype(np.float64)
+    L = lambda a_, b_: float(np.sum(dY * oracle.layer(S, a_, b_, x)))
+    base = L(ad, bd)
+    for k, n in [(0, 0), (1, 5), (2, N - 1)]:
+        a2 = ad.copy(); a2[k, n] += 1.0
+        assert L(a2, bd) - base == pytest.approx(ga[k, n], rel=1e-9, abs=1e-9)
+    for k, j in [(0, 3), (1, K - 1), (2, 40)]:
+        b2 = bd.copy(); b2[k, j] += 1.0
+        assert L(ad, b2) - base == pytest.approx(gb[k, j], rel=1e-9, abs=1e-9)
+
+
+def test_scale_grads_hand_case():
+    # N=1, K=2, one path: W_hat = a*[s0*b0, s1*b1]; G = [g0, g1]
+    S = np.array([[[1, -1]]], dtype=np.int8)
+    a = np.array([[2.0]]); b = np.array([[3.0, 5.0]])
+    G = np.array([[7.0, 11.0]])
+    ga, gb = oracle.scale_grads(G, S, a, b)
+    assert ga[0, 0] == 7 * 3 - 11 * 5              # -34
+    np.testing.assert_array_equal(gb[0], [7 * 2, -11 * 2])
