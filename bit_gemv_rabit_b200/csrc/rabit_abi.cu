@@ -177,6 +177,29 @@ int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, i
                                             scratch, fault, timeout_ns, debug));
 }
 
+size_t rabit_scale_grads_workspace_bytes(int N, int K, int P) {
+    if (N < 1 || K < 1 || P < 1) return 0;
+    return rabit::scale_grads_workspace_bytes(N, K, P);
+}
+
+int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed, const float *a, const float *b,
+                      int N, int K, int P, float *grad_a, float *grad_b, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    if (!G || !packed || !a || !b || !grad_a || !grad_b) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || P < 1 || ldg < K) return RABIT_ERR_SHAPE;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16) || !aligned(G, 4) || !aligned(grad_a, 4) || !aligned(grad_b, 4))
+        return RABIT_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < rabit::scale_grads_workspace_bytes(N, K, P))
+        return RABIT_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    int st = device_ctx(stream, ctx, nullptr);
+    if (st != RABIT_OK) return st;
+    return finish_launch(rabit::launch_scale_grads(ctx, G, ldg, packed, a, b, N, K, P, grad_a, grad_b,
+                                                   workspace));
+}
+
 int rabit_read_fault(void *stream, uint32_t *flags, int clear) {
     rabit::LaunchCtx ctx;
     uint32_t *fault = nullptr;

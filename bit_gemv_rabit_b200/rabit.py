@@ -29,6 +29,8 @@ SIGNATURES = [
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_gemm_noalloc", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p]),
+    ("rabit_scale_grads_workspace_bytes", _sz, [_i, _i, _i]),
+    ("rabit_scale_grads", _i, [_p, _i, _p, _p, _p, _i, _i, _i, _p, _p, _p, _sz, _p]),
     ("rabit_read_fault", _i, [_p, ctypes.POINTER(ctypes.c_uint32), _i]),
     ("rabit_last_cuda_error", _i, []),
     ("rabit_status_string", ctypes.c_char_p, [_i]),
@@ -133,6 +135,26 @@ def rabit_gemm_noalloc(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N
                                      x.stride(0), _dptr(y), y.stride(0), _stream(stream)),
            "rabit_gemm_noalloc")
     return y
+
+
+def rabit_scale_grads_workspace_bytes(N: int, K: int, P: int = 2) -> int:
+    return int(load().rabit_scale_grads_workspace_bytes(N, K, P))
+
+
+def rabit_scale_grads(G: torch.Tensor, packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor,
+                      N: int, K: int, grad_a: torch.Tensor, grad_b: torch.Tensor,
+                      workspace: torch.Tensor, P: int = 2, stream=None):
+    """G [N][K] fp32 (pitch G.stride(0)) = dL/dW_hat; grad_a [P][N], grad_b [P][K] fp32 out."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().rabit_scale_grads(_dptr(G), G.stride(0), _dptr(packed), _dptr(a), _dptr(b), N, K, P,
+                                    _dptr(grad_a), _dptr(grad_b), _dptr(workspace), ws_bytes,
+                                    _stream(stream)), "rabit_scale_grads")
+    return grad_a, grad_b
+
+
+def alloc_scale_grads_workspace(N: int, K: int, P: int = 2, device=None) -> torch.Tensor:
+    return torch.empty(rabit_scale_grads_workspace_bytes(N, K, P), dtype=torch.uint8,
+                       device=device or "cuda")
 
 
 def rabit_read_fault(clear: bool = True, stream=None) -> int:

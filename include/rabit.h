@@ -164,6 +164,28 @@ RABIT_API int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const f
                                  int ldy, void *stream);
 
 /*
+ * rabit_scale_grads -- backward of the layer's scales for a given G = dL/dW_hat (the QAT
+ * backward of sec. 4.2: the shared weight takes G unchanged, the signs are held fixed, and
+ * the learnable scales get the chain rule of sec. 4.1's W_hat = sum_k a_k (.) S_k (.) b_k;
+ * the page text loses the update formula, so the plain chain rule is taken):
+ *     grad_a[k][n] = sum_j G[n][j] * S_k[n][j] * b[k][j]
+ *     grad_b[k][j] = sum_n G[n][j] * a[k][n] * S_k[n][j]
+ * G itself is the dense product dY^T X of the layer's output gradient and input, which the
+ * caller forms (a plain GEMM).  Accumulates in fp32 in a fixed order (deterministic).
+ *   G        [N][ldg] fp32, ldg >= K (input)
+ *   packed   RABIT_LAYOUT_V2 signs of N x K, P paths (input); a [P][N], b [P][K] fp32
+ *   grad_a   [P][N] fp32, grad_b [P][K] fp32 (outputs, fully overwritten)
+ *   workspace  at least rabit_scale_grads_workspace_bytes(N, K, P) bytes, 16-byte aligned,
+ *              caller-owned; no initialisation needed.  Calls sharing it must not overlap.
+ * Errors: INVALID_ARG (null), SHAPE (N, K < 1, ldg < K), UNSUPPORTED (P not 2 or 3),
+ *         ALIGNMENT (packed, G, workspace), WORKSPACE, ARCH, CUDA.
+ */
+RABIT_API size_t rabit_scale_grads_workspace_bytes(int N, int K, int P);
+RABIT_API int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed, const float *a,
+                                const float *b, int N, int K, int P, float *grad_a, float *grad_b,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * rabit_read_fault -- synchronise `stream` and read the current device's fault word
  * (bit set by a kernel whose bounded wait expired).  Returns RABIT_OK when no fault is
  * recorded, RABIT_ERR_TIMEOUT when one is, RABIT_ERR_CUDA on a CUDA failure.  `flags`

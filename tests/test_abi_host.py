@@ -108,6 +108,22 @@ def test_gemm_validation(lib):
     assert f(*args(ws=FAKE + 16)) == ALIGN          # workspace 256-byte alignment
 
 
+def test_scale_grads_validation(lib):
+    f = lib.rabit_scale_grads
+    need = lib.rabit_scale_grads_workspace_bytes(8, 16, 2)
+    assert need == 2 * (1 * 8 + 1 * 16) * 4          # one column tile, one row block
+    args = lambda **kw: [P(kw.get("G", FAKE)), kw.get("ldg", 16), P(kw.get("packed", FAKE)), P(FAKE), P(FAKE),
+                         kw.get("N", 8), kw.get("K", 16), kw.get("P", 2), P(FAKE), P(FAKE),
+                         P(kw.get("ws", FAKE)), kw.get("wsb", need), None]
+    assert f(*args(G=0)) == INVALID
+    assert f(*args(ldg=15)) == SHAPE
+    assert f(*args(N=0)) == SHAPE
+    assert f(*args(P=4)) == UNSUP
+    assert f(*args(packed=FAKE + 4)) == ALIGN
+    assert f(*args(wsb=need - 1)) == WS
+    assert f(*args(ws=FAKE + 4)) == ALIGN
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="valid arguments would launch on a GPU")
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
     st = lib.rabit_derive_pack(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None)
