@@ -333,19 +333,19 @@ prep_x_kernel(const uint16_t *__restrict__ x, int ldx, const float *__restrict__
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+}  // namespace
+
+void *tensor_map_encode_entry() {
+    static void *fn = nullptr;
     if (!fn) {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+            fn = ptr;
     }
     return fn;
 }
-
-}  // namespace
 
 // Scratch for rabit_gemm_noalloc: a fixed buffer in the library's device image, so callers
 // that may not allocate device memory can still run the GEMM.  In host code this name is
@@ -404,7 +404,7 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     }
 
     // 2. Tensor map over the workspace viewed as [P][M][Kp] fp16.
-    auto encode = get_encode_fn();
+    auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap tmap;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(P)};

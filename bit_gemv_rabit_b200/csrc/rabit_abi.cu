@@ -194,10 +194,11 @@ int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed, const flo
         return RABIT_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return RABIT_ERR_ALIGNMENT;
     rabit::LaunchCtx ctx;
-    int st = device_ctx(stream, ctx, nullptr);
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
     return finish_launch(rabit::launch_scale_grads(ctx, G, ldg, packed, a, b, N, K, P, grad_a, grad_b,
-                                                   workspace));
+                                                   workspace, fault, wait_timeout_ns()));
 }
 
 int rabit_read_fault(void *stream, uint32_t *flags, int clear) {

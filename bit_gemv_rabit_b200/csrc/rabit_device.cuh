@@ -22,6 +22,7 @@ enum : uint32_t {
     FAULT_GEMM_WAIT_EPILOGUE = 1u << 3,
     FAULT_GEMM_DRAIN = 1u << 4,
     FAULT_GEMV_WAIT_COPY = 1u << 5,
+    FAULT_SCALE_GRADS_WAIT = 1u << 7,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -100,6 +101,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
         "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// 2-D tiled load (no multicast) into CTA shared memory, completion via mbarrier tx-count.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1)
         : "memory");
 }
 

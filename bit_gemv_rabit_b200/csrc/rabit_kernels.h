@@ -26,10 +26,13 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
                         const float *b, int N, int K, int P, const void *x, bool x_bf16, int batch,
                         int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns);
 
+// The driver's cuTensorMapEncodeTiled (as a PFN_cuTensorMapEncodeTiled_v12000), or null.
+void *tensor_map_encode_entry();
+
 size_t scale_grads_workspace_bytes(int N, int K, int P);
 cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, const uint32_t *packed,
                                const float *a, const float *b, int N, int K, int P, float *grad_a,
-                               float *grad_b, void *workspace);
+                               float *grad_b, void *workspace, uint32_t *fault_word, uint64_t timeout_ns);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
 // Device address and size of the library's fixed GEMM scratch buffer (rabit_gemm_noalloc).
