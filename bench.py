@@ -350,6 +350,32 @@ def bench_gemv_three_path(rabit, device, alu_peak):
             "note": "3 sign words + 1 padding word per group in HBM; algorithmic bytes count the 3 signs"}
 
 
+def bench_scale_grads(rabit, device, hbm_peak):
+    """QAT backward of the scales on the Llama-3-70B MLP shape (G = dL/dW_hat fp32 28672x8192):
+    rabit_scale_grads reads G and the packed signs once (HBM-bound)."""
+    spec = inputs.WORKLOADS["llama3_70b_mlp_qat_m4096"]
+    name, N, K = spec["set"][0]
+    seed = inputs.seed_for(spec["cfg"], 0)
+    W = inputs.weight(seed, N, K, sigma=spec["sigma"])
+    a, b = inputs.scales(seed, W)
+    at, bt = torch.from_numpy(a).to(device), torch.from_numpy(b).to(device)
+    packed = rabit.alloc_packed(N, K, device=device)
+    rabit.rabit_derive_pack(torch.from_numpy(W).to(device), at, bt, packed)
+    del W
+    G = torch.empty((N, K), device=device).normal_(generator=torch.Generator(device=device).manual_seed(seed))
+    ga, gb = torch.empty((2, N), device=device), torch.empty((2, K), device=device)
+    ws = rabit.alloc_scale_grads_workspace(N, K, 2, device=device)
+    g = capture_graph(lambda: rabit.rabit_scale_grads(G, packed, at, bt, N, K, ga, gb, ws))
+    steps = 20
+    ms = timed_replays([g], steps, 3, None, device)
+    byts = N * K * 4 + 2 * N * (((K + 127) // 128) * 128) // 8 + 4 * 2 * (N + K) * 2
+    gbs = byts * steps / (ms * 1e-3) / 1e9
+    return {"workload": "llama3_70b_mlp_scale_grads_28672x8192", "value": round(gbs, 1), "unit": "GB/s",
+            "us_per_call": round(ms / steps * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4)}}
+
+
 def bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained):
     """Llama-3-70B MLP QAT forward: derive_pack of W (fp32 28672x8192) then GEMM at M=4096."""
     spec = inputs.WORKLOADS["llama3_70b_mlp_qat_m4096"]
@@ -597,6 +623,8 @@ def run_ours(args, rank, world, local, dist):
         line.update(bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained))
         torch.cuda.empty_cache()
         line["gemv_3path"] = bench_gemv_three_path(rabit, device, alu_peak)
+        torch.cuda.empty_cache()
+        line["scale_grads"] = bench_scale_grads(rabit, device, hbm_peak)
         torch.cuda.empty_cache()
         prepare_oracle_inputs(base, spec)
         line["cpu_baseline"] = cpu_baseline(base, 1)
