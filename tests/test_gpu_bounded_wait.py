@@ -1,9 +1,9 @@
 """A device wait that runs out is reported, not hung on.
 
 The GEMM's test switch RABIT_TEST_SKIP_ONE_ARRIVE makes the expansion warps skip their first
-arrival, so the MMA warp's bounded wait on that stage expires (after RABIT_WAIT_TIMEOUT_MS).
-The kernel then drains its in-flight copies, frees tensor memory and returns; the host reads
-RABIT_ERR_TIMEOUT with the wait's fault bit, and the next call on the same context is
+arrival, so a bounded wait that depends on it expires (after RABIT_WAIT_TIMEOUT_MS).  The
+kernel then drains its in-flight copies, frees tensor memory and returns; the host reads
+RABIT_ERR_TIMEOUT with a GEMM wait's fault bit, and the next call on the same context is
 correct.  No GPU fault is involved: the failure is a missing arrival that a flag withholds.
 """
 import ctypes
@@ -18,7 +18,10 @@ from bit_gemv_rabit_b200 import rabit
 
 pytestmark = pytest.mark.gpu
 
-FAULT_GEMM_WAIT_MMA = 1 << 1
+# the GEMM's wait bits: TMA producer, MMA issuer, expansion, epilogue.  Every one of them
+# ends up waiting on the withheld arrival; whichever runs out first records its bit and the
+# others see the abort flag.
+FAULT_GEMM_WAITS = (1 << 0) | (1 << 1) | (1 << 2) | (1 << 3)
 RABIT_ERR_TIMEOUT = -8
 
 
@@ -58,7 +61,7 @@ def test_gemm_wait_expiry_is_reported_and_the_context_survives(monkeypatch):
     st = rabit.load().rabit_read_fault(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
                                         ctypes.byref(flags), 1)
     assert st == RABIT_ERR_TIMEOUT
-    assert flags.value & FAULT_GEMM_WAIT_MMA
+    assert flags.value & FAULT_GEMM_WAITS
     monkeypatch.delenv("RABIT_TEST_SKIP_ONE_ARRIVE")
     monkeypatch.delenv("RABIT_WAIT_TIMEOUT_MS")
     # the same context runs the same call correctly afterwards
