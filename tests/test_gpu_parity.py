@@ -207,6 +207,23 @@ def test_gemm_matches_oracle(N, K, M):
     assert err <= TOL_BF16, err
 
 
+def test_gemm_more_tiles_than_sms_matches_oracle():
+    # 16 x 10 = 160 tiles on a 148-SM part: a second, partial round of the persistent tile
+    # loop; every output is compared.
+    N, K, M = 2048, 512, 2560
+    W = inputs.weight(171, N, K)
+    a, b = inputs.scales(171, W)
+    x = inputs.activations(171, M, K, channel_outlier_frac=0.01)
+    at, bt = dev(a), dev(b)
+    packed = rabit.alloc_packed(N, K)
+    rabit.rabit_derive_pack(dev(W), at, bt, packed)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    rabit.rabit_gemm(packed, at, bt, N, K, bf16_dev(x), y, rabit.alloc_gemm_workspace(N, K, 2, M))
+    torch.cuda.synchronize()
+    ref = oracle.layer(oracle.derive_signs(W, a, b), a, b, x)
+    assert normwise(y.cpu().numpy().astype(np.float64), ref) <= TOL_BF16
+
+
 def test_gemm_matches_gemv_bitwise_inputs():
     # The two decode/prefill paths compute the same layer: compare them on one input.
     N, K, M = 256, 1024, 16
