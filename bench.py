@@ -305,6 +305,42 @@ def bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained):
                          "frac_of_nominal_fp8_dense_4500": round(tflops / 4500.0, 4)}}
 
 
+def bench_decode_sweep(rabit, device, alu_peak, hbm_peak):
+    """Llama-3-8B-shaped decode set (q 4096x4096, k/v 1024x4096, gate/up 14336x4096, down
+    4096x14336, 0.1% x20 weight outliers) at batch 1, 4, 8 and 16: microseconds per set and per
+    layer, three rotated copies of the packed weights (more than L2)."""
+    spec = inputs.WORKLOADS["llama3_8b_decode"]
+    out = {"workload": "llama3_8b_decode", "copies": 3, "by_batch": {}}
+    Bmax = max(spec["batches"])
+    base = [make_layer(rabit, spec, idx, name, N, K, device, Bmax)
+            for idx, (name, N, K) in enumerate(spec["set"])]
+    sets = [base] + [[dict(L, packed=L["packed"].clone()) for L in base] for _ in range(2)]
+    torch.cuda.synchronize()
+    sign = sign_bytes(base)
+    for B in spec["batches"]:
+        def step_fn(layers, B=B):
+            def f():
+                for L in layers:
+                    rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"][:B], L["y"][:B])
+            return f
+
+        graphs = [capture_graph(step_fn(ls)) for ls in sets]
+        steps = 600
+        ms = timed_replays(graphs, steps, 30, None, device)
+        us = ms / steps * 1e3
+        byts = decode_bytes(base, batch=B)
+        out["by_batch"][str(B)] = {
+            "us_per_set": round(us, 2), "us_per_layer": round(us / len(base), 2),
+            "GB_per_s": round(byts / (us * 1e-6) / 1e9, 1),
+            "hbm_frac": round(byts / (us * 1e-6) / 1e9 / hbm_peak, 4),
+            # the dp2a pipe applies B sign bits per weight bit at batch B
+            "alu_frac": round(B * sign / (us * 1e-6) / 1e9 / alu_peak, 4)}
+        del graphs
+    del sets, base
+    torch.cuda.empty_cache()
+    return out
+
+
 def warm_launch_us(rabit, layers, device):
     """Microseconds per launch of each distinct shape, re-reading the same weights 200 times
     in a graph (L2-resident after the first launch: the warm-cache setting of the pages'
@@ -625,6 +661,8 @@ def run_ours(args, rank, world, local, dist):
         line["gemv_3path"] = bench_gemv_three_path(rabit, device, alu_peak)
         torch.cuda.empty_cache()
         line["scale_grads"] = bench_scale_grads(rabit, device, hbm_peak)
+        torch.cuda.empty_cache()
+        line["decode_batch_sweep"] = bench_decode_sweep(rabit, device, alu_peak, hbm_peak)
         torch.cuda.empty_cache()
         prepare_oracle_inputs(base, spec)
         line["cpu_baseline"] = cpu_baseline(base, 1)
