@@ -99,3 +99,26 @@ def test_gemm_workloads_full_size(workload):
         ref = oracle.layer(S_rows, a, b, x, rows=rows, N=N)
         err = normwise(y.cpu().numpy()[:, rows].astype(np.float64), ref)
         assert err <= TOL, (name, err)
+
+
+def test_three_path_decode_set_full_size():
+    """The 3-bit variant on the Llama-2-7B decode set at batch 1 (sampled rows)."""
+    spec = inputs.WORKLOADS["llama2_7b_decode_b1"]
+    for idx, (name, N, K) in enumerate(spec["set"]):
+        seed = inputs.seed_for(spec["cfg"], idx)
+        W = inputs.weight(seed, N, K, sigma=spec["sigma"])
+        a, b = inputs.scales(seed, W, P=3)
+        rows = sample_rows(N, seed, count=24)
+        packed = rabit.alloc_packed(N, K, P=3)
+        at, bt = torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()
+        rabit.rabit_derive_pack(torch.from_numpy(W).cuda(), at, bt, packed, P=3)
+        x = inputs.activations(seed, 1, K)
+        y = torch.empty((1, N), device="cuda")
+        rabit.rabit_gemv(packed, at, bt, N, K, bf16_dev(x), y, P=3)
+        torch.cuda.synchronize()
+        per_row = oracle.packed_words(1, K, 3)
+        S_rows = np.concatenate([oracle.derive_signs(W, a, b, P=3, rows=(int(r), int(r) + 1)) for r in rows], axis=1)
+        np.testing.assert_array_equal(packed.cpu().numpy().reshape(N, per_row)[rows],
+                                      oracle.pack(S_rows).reshape(len(rows), per_row))
+        ref = oracle.layer(S_rows, a, b, x, rows=rows, N=N)
+        assert normwise(y.cpu().numpy()[:, rows].astype(np.float64), ref) <= TOL, name
