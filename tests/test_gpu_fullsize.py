@@ -122,3 +122,20 @@ def test_three_path_decode_set_full_size():
                                       oracle.pack(S_rows).reshape(len(rows), per_row))
         ref = oracle.layer(S_rows, a, b, x, rows=rows, N=N)
         assert normwise(y.cpu().numpy()[:, rows].astype(np.float64), ref) <= TOL, name
+
+
+def test_gemv_several_passes_and_batch_rows():
+    """28672 x 8192 leaves each CTA 194 rows of 2 KiB: more than its shared memory holds, so
+    the rows go through several passes, each reused by 3 batch rows (sampled rows)."""
+    N, K, B = 28672, 8192, 3
+    seed = 777
+    W = inputs.weight(seed, N, K, sigma=0.015)
+    a, b = inputs.scales(seed, W)
+    rows = sample_rows(N, seed, count=24)
+    packed, S_rows = derive_and_check(W, a, b, rows)
+    x = inputs.activations(seed, B, K)
+    y = torch.empty((B, N), device="cuda")
+    rabit.rabit_gemv(packed, torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), N, K, bf16_dev(x), y)
+    torch.cuda.synchronize()
+    ref = oracle.layer(S_rows, a, b, x, rows=rows, N=N)
+    assert normwise(y.cpu().numpy()[:, rows].astype(np.float64), ref) <= TOL
