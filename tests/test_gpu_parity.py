@@ -126,7 +126,7 @@ GEMV_SHAPES = [(1, 1), (32, 128), (33, 129), (96, 1000), (300, 520), (1024, 4096
 
 
 @pytest.mark.parametrize("N,K", GEMV_SHAPES)
-@pytest.mark.parametrize("batch", [1, 3, 16])
+@pytest.mark.parametrize("batch", [1, 2, 3, 8, 16])
 def test_gemv_bf16_matches_oracle(N, K, batch):
     W, a, b = make_layer(200 + N, N, K)
     S = oracle.derive_signs(W, a, b)
@@ -151,6 +151,29 @@ def test_gemv_fp32_matches_oracle(N, K, batch):
     torch.cuda.synchronize()
     ref = oracle.layer(S, a, b, x)
     assert normwise(y.cpu().numpy().astype(np.float64), ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("P", [2, 3])
+@pytest.mark.parametrize("N,K,batch", [(300, 520, 2), (300, 520, 7), (1024, 4096, 4), (4096, 4096, 6),
+                                       (1000, 1000, 16)])
+def test_gemv_each_batch_row_matches_oracle(N, K, batch, P):
+    """Batch rows of magnitudes 2^-6 .. 2^+6 apart: every row is checked on its own, so a row
+    scaled with another row's z scale, or left unwritten, fails."""
+    W, a, b = make_layer(400 + N + batch, N, K)
+    a3, b3 = inputs.scales(400 + N, W, P=P)
+    S = oracle.derive_signs(W, a3, b3, P=P)
+    x = inputs.activations(401 + K, batch, K)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    xf = xf * np.float32(2.0) ** np.array([(3 * beta) % 13 - 6 for beta in range(batch)],
+                                          np.float32)[:, None]
+    xb = (xf.view(np.uint32) >> 16).astype(np.uint16)      # power-of-two scaling is exact in bf16
+    y = torch.full((batch, N), float("nan"), device="cuda")
+    rabit.rabit_gemv(dev(oracle.pack(S)), dev(a3), dev(b3), N, K, bf16_dev(xb), y, P=P)
+    torch.cuda.synchronize()
+    ref = oracle.layer(S, a3, b3, xb)
+    yh = y.cpu().numpy().astype(np.float64)
+    for beta in range(batch):
+        assert normwise(yh[beta], ref[beta]) <= TOL_BF16, beta
 
 
 def test_gemv_pitched_io():
