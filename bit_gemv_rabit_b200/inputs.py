@@ -16,6 +16,10 @@ Recipe (one function per workload item):
     first-path residual without computing that residual here.
   * x ~ N(0, 1) rounded to bf16 (round-to-nearest-even), [B][K]; optionally a fraction of
     the K channels (the same channels for every token) multiplied by a factor.
+  * calibration statistics for the initialisation's preconditioning: s_in [K] stands for
+    the per-channel max |activation| (log-normal, sigma 0.5, with 1% of the channels x10)
+    and s_out [N] for the per-row max |output gradient| (log-normal, sigma 0.3); each is
+    divided by its mean.  No calibration data is used.
 """
 from __future__ import annotations
 
@@ -85,6 +89,18 @@ def activations(seed: int, B: int, K: int, channel_outlier_frac: float = 0.0,
     if dtype == "f32":
         return x
     raise ValueError(dtype)
+
+
+def calibration_stats(seed: int, N: int, K: int, outlier_frac: float = 0.01,
+                      outlier_scale: float = 10.0) -> tuple[np.ndarray, np.ndarray]:
+    """(s_in [K], s_out [N]) fp32, positive, each with mean 1 (see module recipe)."""
+    rng = rng_for(seed + 15485863)
+    s_in = np.exp(0.5 * rng.standard_normal(K))
+    if outlier_frac > 0.0:
+        count = max(1, int(round(outlier_frac * K)))
+        s_in[rng.choice(K, size=count, replace=False)] *= outlier_scale
+    s_out = np.exp(0.3 * rng.standard_normal(N))
+    return (s_in / s_in.mean()).astype(np.float32), (s_out / s_out.mean()).astype(np.float32)
 
 
 # Workload shapes, named by what they are.  Each entry: (name, N, K).

@@ -1,0 +1,142 @@
+"""Pins of the float64 initialisation oracle (oracle/svid.py) against facts fixed outside it.
+
+  * a signed rank-1 matrix g0 (.) S0 (.) h0 is recovered exactly, with and without
+    preconditioning (pins the sign rule, the rank-1 step, the preconditioning direction and
+    the map-back exponents)                                                 -> svid_init
+  * the objective ||W' - sum_i What_i||_F never increases over the (t, i) updates (each update
+    is optimal for its path given the others: the sign of the residual, then Eckart-Young
+    for |R|)                                                                 -> svid_init
+  * the rank-1 step against an independent power iteration written here     -> rank1_abs
+  * the reconstruction does not depend on the normalisation of s_in, s_out   -> svid_init
+  * the last update is locally optimal: perturbing its scales raises the error -> svid_init
+  * a planted mistake in the map-back (wrong exponent sign) is caught by the invariance pin
+Source: "RaBiT: Residual-Aware Binarization Training for Accurate and Efficient LLMs",
+sec. 4.3 "Stable Initialization for Functional Preservation" (Iterative Residual SVID,
+I/O Channel Importance-Scaled Preconditioning), Appendix F.3 (iteration 1 is greedy).
+"""
+import numpy as np
+import pytest
+
+from oracle import svid as osvid
+from bit_gemv_rabit_b200 import inputs
+
+ALPHA_IN, ALPHA_OUT = 0.8, 0.65   # the pages' Table 11 intensities for Llama2-7B, 2 bits
+
+
+def signed_rank1(seed, N, K):
+    rng = np.random.default_rng(seed)
+    g0 = rng.uniform(0.5, 2.0, N)
+    h0 = rng.uniform(0.5, 2.0, K)
+    S0 = np.where(rng.random((N, K)) < 0.5, -1, 1).astype(np.int8)
+    return g0, S0, h0
+
+
+@pytest.mark.parametrize("P", [2, 3])
+def test_signed_rank1_is_recovered_exactly(P):
+    N, K = 24, 40
+    g0, S0, h0 = signed_rank1(1, N, K)
+    W = g0[:, None] * S0 * h0[None, :]
+    ones_k, ones_n = np.ones(K), np.ones(N)
+    S, a, b = osvid.svid_init(W, ones_k, ones_n, ALPHA_IN, ALPHA_OUT, P=P, T=3)
+    np.testing.assert_array_equal(S[0], S0)
+    np.testing.assert_allclose(np.outer(a[0], b[0]), np.outer(g0, h0), rtol=1e-12)
+    for i in range(1, P):           # the residual is 0 up to the rounding of the first path
+        assert np.max(np.outer(a[i], b[i])) <= 1e-12 * np.max(np.abs(W))
+    np.testing.assert_allclose(osvid.reconstruct(S, a, b), W, rtol=1e-12, atol=0)
+
+
+def test_preconditioned_signed_rank1_maps_back_exactly():
+    """W = s_out^-alpha_out (.) (g0 S0 h0) (.) s_in^-alpha_in makes W' signed rank-1; the scales
+    mapped back must rebuild W itself."""
+    N, K = 30, 52
+    g0, S0, h0 = signed_rank1(2, N, K)
+    s_in, s_out = inputs.calibration_stats(3, N, K)
+    si, so = s_in.astype(np.float64) ** ALPHA_IN, s_out.astype(np.float64) ** ALPHA_OUT
+    W = (g0[:, None] * S0 * h0[None, :]) / so[:, None] / si[None, :]
+    S, a, b = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=2, T=2)
+    np.testing.assert_array_equal(S[0], S0)
+    np.testing.assert_allclose(osvid.reconstruct(S, a, b), W, rtol=1e-11, atol=0)
+    np.testing.assert_allclose(np.outer(a[0], b[0]), W * S0, rtol=1e-11)
+
+
+@pytest.mark.parametrize("P,precond", [(2, False), (2, True), (3, True)])
+def test_objective_never_increases(P, precond):
+    N, K = 48, 80
+    W = inputs.weight(5, N, K, outlier_frac=0.01)
+    s_in, s_out = inputs.calibration_stats(5, N, K) if precond else (np.ones(K), np.ones(N))
+    S, a, b, hist = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=P, T=8, history=True)
+    assert len(hist) == 1 + 8 * P
+    h = np.array(hist)
+    assert np.all(np.diff(h) <= 1e-12 * h[0])
+    assert h[-1] < h[P]           # iterating improves on the greedy (t = 1) decomposition here
+    Wp = osvid.precondition(W, s_in, s_out, ALPHA_IN, ALPHA_OUT)
+    si = np.asarray(s_in, np.float64) ** ALPHA_IN
+    so = np.asarray(s_out, np.float64) ** ALPHA_OUT
+    Wh = osvid.reconstruct(S, a * so[None, :], b * si[None, :])
+    assert abs(np.linalg.norm(Wp - Wh) - h[-1]) <= 1e-10 * h[0]
+
+
+def test_rank1_step_matches_power_iteration():
+    rng = np.random.default_rng(7)
+    R = rng.standard_normal((37, 61)) * np.exp(rng.standard_normal(61))[None, :]
+    sigma, u, v = osvid.rank1_abs(R)
+    A = np.abs(R)
+    x = np.ones(61)
+    for _ in range(2000):
+        y = A @ x
+        x = A.T @ y
+        x /= np.linalg.norm(x)
+    y = A @ x
+    sig_pi = np.linalg.norm(y)
+    assert abs(sigma - sig_pi) <= 1e-10 * sigma
+    np.testing.assert_allclose(v, x, atol=1e-9)
+    np.testing.assert_allclose(u, y / sig_pi, atol=1e-9)
+    assert np.all(u >= 0) and np.all(v >= 0)
+
+
+def test_reconstruction_is_independent_of_stat_normalisation():
+    N, K = 40, 72
+    W = inputs.weight(9, N, K)
+    s_in, s_out = inputs.calibration_stats(9, N, K)
+    S1, a1, b1 = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=2, T=4)
+    S2, a2, b2 = osvid.svid_init(W, 7.0 * s_in, 0.3 * s_out, ALPHA_IN, ALPHA_OUT, P=2, T=4)
+    np.testing.assert_array_equal(S1, S2)
+    # the same iteration on inputs scaled by constants: equal up to rounding
+    np.testing.assert_allclose(osvid.reconstruct(S2, a2, b2), osvid.reconstruct(S1, a1, b1),
+                               rtol=1e-6, atol=0)
+
+
+def test_last_update_is_locally_optimal():
+    N, K = 32, 64
+    W = inputs.weight(11, N, K)
+    s_in, s_out = inputs.calibration_stats(11, N, K)
+    S, a, b = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=2, T=5)
+    Wp = osvid.precondition(W, s_in, s_out, ALPHA_IN, ALPHA_OUT)
+    si = np.asarray(s_in, np.float64) ** ALPHA_IN
+    so = np.asarray(s_out, np.float64) ** ALPHA_OUT
+    g, h = a * so[None, :], b * si[None, :]
+    base = np.linalg.norm(Wp - osvid.reconstruct(S, g, h))
+    rng = np.random.default_rng(12)
+    for _ in range(20):
+        g2, h2 = g.copy(), h.copy()
+        g2[1] *= 1 + 1e-3 * rng.standard_normal(N)
+        h2[1] *= 1 + 1e-3 * rng.standard_normal(K)
+        assert np.linalg.norm(Wp - osvid.reconstruct(S, g2, h2)) >= base * (1 - 1e-12)
+
+
+def test_planted_map_back_mistake_is_caught(monkeypatch):
+    """The invariance pin catches a map-back that multiplies by s^alpha instead of dividing."""
+    N, K = 20, 36
+    W = inputs.weight(13, N, K)
+    s_in, s_out = inputs.calibration_stats(13, N, K)
+    real = osvid.svid_init
+
+    def planted(W, s_in, s_out, alpha_in, alpha_out, **kw):
+        S, a, b = real(W, s_in, s_out, alpha_in, alpha_out, **kw)
+        so = np.asarray(s_out, np.float64) ** alpha_out
+        si = np.asarray(s_in, np.float64) ** alpha_in
+        return S, a * so[None, :] ** 2, b * si[None, :] ** 2
+    monkeypatch.setattr(osvid, "svid_init", planted)
+    S1, a1, b1 = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=2, T=2)
+    S2, a2, b2 = osvid.svid_init(W, 7.0 * s_in, 0.3 * s_out, ALPHA_IN, ALPHA_OUT, P=2, T=2)
+    assert not np.allclose(osvid.reconstruct(S2, a2, b2), osvid.reconstruct(S1, a1, b1), rtol=1e-6)
