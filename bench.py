@@ -14,7 +14,8 @@ The printed JSON line carries the metric (packed-weight HBM GB/s of the decode p
 roofline of the GEMV kernel, the SM clocks seen during the timed region, an end-to-end
 figure through the public Python API with host copies, and, on rank 0 with one GPU, the
 secondary measurements of the same metric string (rabit_gemm TFLOP/s at M=2048 on the
-Llama-3-8B MLP shapes, rabit_derive_pack GB/s and the Llama-3-70B MLP QAT step) plus the
+Llama-3-8B MLP shapes, rabit_derive_pack GB/s, the Llama-3-70B MLP QAT step, the scale
+gradients and the Iterative Residual SVID initialisation of a 4096x4096 layer) plus the
 float64 oracle timed on a bounded sample as the CPU baseline.
 
 --impl reference times the float64 CPU oracle (the reference arm of this repository) on the
@@ -412,6 +413,54 @@ def bench_scale_grads(rabit, device, hbm_peak):
                          "frac": round(gbs / hbm_peak, 4)}}
 
 
+SVID_T, SVID_POWER_ITERS = 20, 40
+SVID_ALPHA_IN, SVID_ALPHA_OUT = 0.8, 0.65   # the pages' Table 11 intensities, Llama2-7B, 2 bits
+
+
+def bench_svid_init(rabit, device, hbm_peak):
+    """Initialisation of one Llama-2-7B q_proj-shaped layer (4096x4096 fp32 W, seeded
+    calibration statistics): Iterative Residual SVID, T = 20, two paths, 40 power steps per
+    update.  Algorithmic bytes per update: the residual pass reads W and writes R (fp32) and
+    the signs; each power step reads R and the two-word packed signs."""
+    spec = inputs.WORKLOADS["llama2_7b_decode_b1"]
+    name, N, K = spec["set"][0]
+    seed = inputs.seed_for(spec["cfg"], 0)
+    W = torch.from_numpy(inputs.weight(seed, N, K, sigma=spec["sigma"])).to(device)
+    s_in, s_out = inputs.calibration_stats(seed, N, K)
+    si, so = torch.from_numpy(s_in).to(device), torch.from_numpy(s_out).to(device)
+    P = 2
+    a, b = torch.empty((P, N), device=device), torch.empty((P, K), device=device)
+    packed = rabit.alloc_packed(N, K, P=P, device=device)
+    ws = rabit.alloc_svid_init_workspace(N, K, P, device=device)
+
+    def run():
+        rabit.rabit_svid_init(W, si, so, SVID_ALPHA_IN, SVID_ALPHA_OUT, a, b, packed, ws, P=P, T=SVID_T,
+                              power_iters=SVID_POWER_ITERS)
+    run()
+    torch.cuda.synchronize()
+    reps = 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nk = N * K
+    sign_bytes = N * (((K + 127) // 128) * 128) // 8
+    per_update = (4 * nk + 4 * nk + (P - 1) * sign_bytes + 3 * sign_bytes
+                  + SVID_POWER_ITERS * (4 * nk + 2 * sign_bytes))
+    byts = SVID_T * P * per_update
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"workload": "llama2_7b_q_proj_4096x4096_svid_init", "T": SVID_T, "P": P,
+            "power_iters": SVID_POWER_ITERS, "ms_per_init": round(ms, 3),
+            "launches_per_init": 2 + SVID_T * P * (1 + 3 * SVID_POWER_ITERS),
+            "value": round(gbs, 1), "unit": "GB/s",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4),
+                         "note": "the 67 MB residual is re-read by every power step and fits in L2"}}
+
+
 def bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained):
     """Llama-3-70B MLP QAT forward: derive_pack of W (fp32 28672x8192) then GEMM at M=4096."""
     spec = inputs.WORKLOADS["llama3_70b_mlp_qat_m4096"]
@@ -661,6 +710,8 @@ def run_ours(args, rank, world, local, dist):
         line["gemv_3path"] = bench_gemv_three_path(rabit, device, alu_peak)
         torch.cuda.empty_cache()
         line["scale_grads"] = bench_scale_grads(rabit, device, hbm_peak)
+        torch.cuda.empty_cache()
+        line["svid_init"] = bench_svid_init(rabit, device, hbm_peak)
         torch.cuda.empty_cache()
         line["decode_batch_sweep"] = bench_decode_sweep(rabit, device, alu_peak, hbm_peak)
         torch.cuda.empty_cache()

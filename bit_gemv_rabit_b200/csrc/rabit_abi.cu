@@ -3,6 +3,7 @@
 // Each entry point validates every argument on the host before anything is enqueued
 // (pure argument checks first, then the device checks), then calls one launcher.  Nothing
 // here computes any part of the layer: all arithmetic runs in the CUDA kernels.
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -199,6 +200,33 @@ int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed, const flo
     if (st != RABIT_OK) return st;
     return finish_launch(rabit::launch_scale_grads(ctx, G, ldg, packed, a, b, N, K, P, grad_a, grad_b,
                                                    workspace, fault, wait_timeout_ns()));
+}
+
+size_t rabit_svid_init_workspace_bytes(int N, int K, int P) {
+    if (N < 1 || K < 1 || (P != 2 && P != 3)) return 0;
+    return rabit::svid_workspace_bytes(N, K, P);
+}
+
+int rabit_svid_init(const float *W, int N, int K, int ldw, int P, int T, int power_iters,
+                    const float *s_in, const float *s_out, float alpha_in, float alpha_out, float *a,
+                    float *b, uint32_t *packed, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!W || !s_in || !s_out || !a || !b || !packed) return RABIT_ERR_INVALID_ARG;
+    if (!std::isfinite(alpha_in) || !std::isfinite(alpha_out)) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || ldw < K || T < 1 || T > RABIT_SVID_MAX_ITERS || power_iters < 1 ||
+        power_iters > RABIT_SVID_MAX_ITERS)
+        return RABIT_ERR_SHAPE;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16) || !aligned(W, 4) || !aligned(s_in, 4) || !aligned(s_out, 4) || !aligned(a, 4) ||
+        !aligned(b, 4))
+        return RABIT_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < rabit::svid_workspace_bytes(N, K, P)) return RABIT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
+    if (st != RABIT_OK) return st;
+    return finish_launch(rabit::launch_svid_init(ctx, W, ldw, N, K, P, T, power_iters, s_in, s_out, alpha_in,
+                                                 alpha_out, a, b, packed, workspace, fault, wait_timeout_ns()));
 }
 
 int rabit_read_fault(void *stream, uint32_t *flags, int clear) {

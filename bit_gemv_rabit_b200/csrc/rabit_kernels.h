@@ -34,6 +34,13 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
                                const float *a, const float *b, int N, int K, int P, float *grad_a,
                                float *grad_b, void *workspace, uint32_t *fault_word, uint64_t timeout_ns);
 
+// Iterative Residual SVID initialisation (svid.cu).
+size_t svid_workspace_bytes(int N, int K, int P);
+cudaError_t launch_svid_init(const LaunchCtx &ctx, const float *W, int ldw, int N, int K, int P, int T,
+                             int power_iters, const float *s_in, const float *s_out, float alpha_in,
+                             float alpha_out, float *a, float *b, uint32_t *packed, void *workspace,
+                             uint32_t *fault_word, uint64_t timeout_ns);
+
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
 // Device address and size of the library's fixed GEMM scratch buffer (rabit_gemm_noalloc).
 cudaError_t gemm_noalloc_scratch(void **ptr, size_t *bytes);

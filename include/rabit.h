@@ -186,6 +186,43 @@ RABIT_API int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * rabit_svid_init -- initialisation of the layer's paths and scales (sec. 4.3 "Stable
+ * Initialization for Functional Preservation"): Iterative Residual SVID on the
+ * importance-preconditioned weight, scales mapped back to the original domain.
+ *     W' = s_out^alpha_out (.) W (.) s_in^alpha_in          (row scale s_out, column scale s_in)
+ *     for t = 1..T, i = 1..P:  R_i = W' - sum_{j != i} What_j   (latest update of each path,
+ *                                                           What_j = 0 before its first)
+ *         B_i = sign(R_i),  g_i' h_i'^T = sigma u v^T, the leading rank-1 part of |R_i|,
+ *         g_i' = sqrt(sigma) u,  h_i' = sqrt(sigma) v,  What_i = g_i' (.) B_i (.) h_i'
+ *     a[i] = g_i' / s_out^alpha_out,   b[i] = h_i' / s_in^alpha_in
+ * SVID is read as the sign-value-independent decomposition (sign plus the best rank-1
+ * approximation of |R|), which the pages cite but do not define.  The leading singular
+ * pair comes from `power_iters` power steps per update (fp32, deterministic order),
+ * warm-started from the path's pair of the previous iteration (uniform vectors at t = 1).
+ * The pages use T = 20.
+ *   W        [N][ldw] fp32, ldw >= K (input)
+ *   s_in [K], s_out [N]  positive fp32 calibration statistics (inputs; the reconstruction
+ *            sum_i a_i (.) B_i (.) b_i does not depend on their normalisation);
+ *            non-positive or non-finite entries give undefined (inf or NaN) outputs
+ *   a [P][N], b [P][K] fp32 (outputs, fully overwritten)
+ *   packed   RABIT_LAYOUT_V2 buffer of N x K, P paths: the final B_i (output, every word
+ *            written, padding included)
+ *   workspace  at least rabit_svid_init_workspace_bytes(N, K, P) bytes (about 4*N*K),
+ *              256-byte aligned, caller-owned, no initialisation needed.  Calls sharing it
+ *              must not overlap.
+ * Enqueues about T * P * (1 + 3 * power_iters) kernels on `stream` and returns.
+ * Errors: INVALID_ARG (null, non-finite alpha), SHAPE (N, K < 1, ldw < K, T or power_iters
+ *         outside 1..RABIT_SVID_MAX_ITERS), UNSUPPORTED (P not 2 or 3), ALIGNMENT (packed,
+ *         workspace), WORKSPACE, ARCH, CUDA.
+ */
+#define RABIT_SVID_MAX_ITERS 1000
+RABIT_API size_t rabit_svid_init_workspace_bytes(int N, int K, int P);
+RABIT_API int rabit_svid_init(const float *W, int N, int K, int ldw, int P, int T, int power_iters,
+                              const float *s_in, const float *s_out, float alpha_in, float alpha_out,
+                              float *a, float *b, uint32_t *packed, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
  * rabit_read_fault -- synchronise `stream` and read the current device's fault word
  * (bit set by a kernel whose bounded wait expired).  Returns RABIT_OK when no fault is
  * recorded, RABIT_ERR_TIMEOUT when one is, RABIT_ERR_CUDA on a CUDA failure.  `flags`

@@ -124,6 +124,30 @@ def test_scale_grads_validation(lib):
     assert f(*args(ws=FAKE + 4)) == ALIGN
 
 
+def test_svid_init_validation(lib):
+    f = lib.rabit_svid_init
+    need = lib.rabit_svid_init_workspace_bytes(8, 16, 2)
+    assert need >= 8 * 16 * 4                         # the residual alone
+    assert lib.rabit_svid_init_workspace_bytes(8, 16, 4) == 0
+    args = lambda **kw: [P(kw.get("W", FAKE)), kw.get("N", 8), kw.get("K", 16), kw.get("ldw", 16), kw.get("P", 2),
+                         kw.get("T", 20), kw.get("iters", 40), P(FAKE), P(FAKE), kw.get("ai", 0.8),
+                         kw.get("ao", 0.65), P(FAKE), P(FAKE), P(kw.get("packed", FAKE)),
+                         P(kw.get("ws", FAKE)), kw.get("wsb", need), None]
+    assert f(*args(W=0)) == INVALID
+    assert f(*args(ai=float("nan"))) == INVALID
+    assert f(*args(ao=float("inf"))) == INVALID
+    assert f(*args(N=0)) == SHAPE
+    assert f(*args(ldw=15)) == SHAPE
+    assert f(*args(T=0)) == SHAPE
+    assert f(*args(T=1001)) == SHAPE
+    assert f(*args(iters=0)) == SHAPE
+    assert f(*args(P=4)) == UNSUP
+    assert f(*args(packed=FAKE + 4)) == ALIGN
+    assert f(*args(wsb=need - 1)) == WS
+    assert f(*args(ws=0)) == WS
+    assert f(*args(ws=FAKE + 16)) == ALIGN
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="valid arguments would launch on a GPU")
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
     st = lib.rabit_derive_pack(P(FAKE), 0, 4, 4, 4, 2, P(FAKE), P(FAKE), P(FAKE), None)
