@@ -65,6 +65,10 @@ def parse_args(argv=None):
     ap.add_argument("--shape", type=int, nargs=3, metavar=("N", "K", "M"), default=(11008, 4096, 1),
                     help="with --profile-kernel: out features, in features, batch/tokens")
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="time the float64 CPU oracle on every workload (no GPU) and exit")
+    ap.add_argument("--gemm-token-sample", type=int, default=8,
+                    help="with --oracle-table: tokens of the GEMM workloads the oracle evaluates")
     return ap.parse_args(argv)
 
 
@@ -530,6 +534,46 @@ def prepare_oracle_inputs(layers, spec):
         L["S_cache"] = oracle.derive_signs(W, a, b)
 
 
+def oracle_table(args):
+    """The float64 oracle timed on every workload, on this host's cores (a CPU baseline
+    only): derive + pack per matrix, the layer at every batch of the decode workloads, and
+    for the GEMM workloads the layer on a sample of tokens, scaled to the full token count
+    (the layer's cost is linear in the tokens) and labelled as such."""
+    import oracle
+    oracle.build()
+    out = {"kind": "oracle", "cores": oracle.num_threads(), "host": "this host's CPU cores",
+           "workloads": {}}
+    for wname, spec in inputs.WORKLOADS.items():
+        rows = []
+        for idx, (name, N, K) in enumerate(spec["set"]):
+            seed = inputs.seed_for(spec["cfg"], idx)
+            W = inputs.weight(seed, N, K, sigma=spec["sigma"], outlier_frac=spec["w_outliers"])
+            a, b = inputs.scales(seed, W)
+            t0 = time.perf_counter()
+            S = oracle.derive_signs(W, a, b)
+            oracle.pack(S)
+            t_derive = time.perf_counter() - t0
+            del W
+            row = {"matrix": f"{name} {N}x{K}", "derive_pack_s": round(t_derive, 3)}
+            gemm = max(spec["batches"]) > 16
+            for B in spec["batches"]:
+                Bs = min(B, args.gemm_token_sample) if gemm else B
+                x = inputs.activations(seed, Bs, K, channel_outlier_frac=spec["x_outliers"])
+                t0 = time.perf_counter()
+                oracle.layer(S, a, b, x)
+                t = time.perf_counter() - t0
+                if gemm:
+                    row[f"layer_m{B}_s"] = round(t * B / Bs, 4)
+                    row["token_sample"] = Bs
+                else:
+                    row[f"layer_b{B}_us"] = round(t * 1e6, 1)
+            rows.append(row)
+            del S
+        out["workloads"][wname] = rows
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     """The float64 CPU oracle as the reference arm: each step is a bounded sample of rows."""
@@ -586,6 +630,8 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------- main
 def main(argv=None):
     args = parse_args(argv)
+    if args.oracle_table:
+        return oracle_table(args)
     rank, world, local, dist = dist_init()
     try:
         if args.profile_kernel:
