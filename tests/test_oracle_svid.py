@@ -10,6 +10,7 @@
   * the reconstruction does not depend on the normalisation of s_in, s_out   -> svid_init
   * the last update is locally optimal: perturbing its scales raises the error -> svid_init
   * a planted mistake in the map-back (wrong exponent sign) is caught by the invariance pin
+  * a hand-worked diagonal weight (closed form for 2 and 3 paths) and the zero weight
 Source: "RaBiT: Residual-Aware Binarization Training for Accurate and Efficient LLMs",
 sec. 4.3 "Stable Initialization for Functional Preservation" (Iterative Residual SVID,
 I/O Channel Importance-Scaled Preconditioning), Appendix F.3 (iteration 1 is greedy).
@@ -74,6 +75,35 @@ def test_objective_never_increases(P, precond):
     so = np.asarray(s_out, np.float64) ** ALPHA_OUT
     Wh = osvid.reconstruct(S, a * so[None, :], b * si[None, :])
     assert abs(np.linalg.norm(Wp - Wh) - h[-1]) <= 1e-10 * h[0]
+
+
+def test_diagonal_weight_hand_case():
+    """W = diag(3, -2, 1), no preconditioning.  |R| of each update is diagonal, so its leading
+    rank-1 part is the largest entry alone: path 1 takes 3 (sigma 3, u = v = e1), path 2 takes
+    -2, path 3 takes 1.  Zero residual entries are +1 (sign rule).  By hand:
+      P = 3: exact, a_i = b_i = sqrt(sigma_i) e_i;
+      P = 2: the entry 1 is left over, ||W - W_hat||_F = 1, at every T (fixed point)."""
+    W = np.diag([3.0, -2.0, 1.0])
+    ones = np.ones(3)
+    S, a, b = osvid.svid_init(W, ones, ones, ALPHA_IN, ALPHA_OUT, P=3, T=1)
+    np.testing.assert_allclose(osvid.reconstruct(S, a, b), W, atol=1e-12)
+    for i, sig in enumerate([3.0, 2.0, 1.0]):
+        e = np.eye(3)[i]
+        np.testing.assert_allclose(a[i], np.sqrt(sig) * e, atol=1e-12)
+        np.testing.assert_allclose(b[i], np.sqrt(sig) * e, atol=1e-12)
+    # -2 is negative in W (path 1) and in R_2 = diag(0, -2, 1) (path 2); R_3 = diag(0, 0, 1)
+    assert S[0][1, 1] == -1 and S[1][1, 1] == -1 and np.sum(S == -1) == 2
+    for T in (1, 2, 5):
+        S2, a2, b2 = osvid.svid_init(W, ones, ones, ALPHA_IN, ALPHA_OUT, P=2, T=T)
+        assert abs(np.linalg.norm(W - osvid.reconstruct(S2, a2, b2)) - 1.0) <= 1e-12
+
+
+def test_zero_weight_gives_zero_scales():
+    """W = 0: every residual is 0, so sigma = 0, the scales are 0 and the signs +1."""
+    N, K = 5, 7
+    s_in, s_out = inputs.calibration_stats(2, N, K)
+    S, a, b = osvid.svid_init(np.zeros((N, K)), s_in, s_out, ALPHA_IN, ALPHA_OUT, P=2, T=3)
+    assert np.all(S == 1) and not np.any(a) and not np.any(b)
 
 
 def test_rank1_step_matches_power_iteration():
