@@ -100,3 +100,21 @@ def test_svid_init_pitched_w_and_repeatability():
     np.testing.assert_array_equal(p1, p2)
     np.testing.assert_array_equal(a1, a2)
     np.testing.assert_array_equal(b1, b2)
+
+
+def test_svid_init_degenerate_cases():
+    """W = 0 gives zero scales and all-+1 signs; W = diag(3, -2, 1) with three paths is
+    rebuilt exactly, a_i = b_i = sqrt(sigma_i) e_i with sigma = 3, 2, 1 (hand-worked in the
+    oracle's pins)."""
+    ones3 = np.ones(3, np.float32)
+    a, b, packed = gpu_init(np.zeros((5, 7), np.float32), *inputs.calibration_stats(2, 5, 7), P=2, T=3)
+    assert not np.any(a) and not np.any(b)
+    assert np.all(oracle.unpack(packed, 5, 7, P=2) == 1)
+    W = np.diag([3.0, -2.0, 1.0]).astype(np.float32)
+    a, b, packed = gpu_init(W, ones3, ones3, P=3, T=1)
+    S = oracle.unpack(packed, 3, 3, P=3)
+    np.testing.assert_array_equal(S[0], np.where(W < 0, -1, 1))
+    assert fro(osvid.reconstruct(S, a, b), W.astype(np.float64)) <= 1e-5
+    for i, sig in enumerate([3.0, 2.0, 1.0]):
+        np.testing.assert_allclose(a[i], np.sqrt(sig) * np.eye(3)[i], atol=1e-5)
+        np.testing.assert_allclose(b[i], np.sqrt(sig) * np.eye(3)[i], atol=1e-5)
