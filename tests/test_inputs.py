@@ -32,3 +32,19 @@ def test_generators_are_seeded_and_shaped():
     xf = inputs.bf16_to_f32(x)
     big = np.abs(xf).max(axis=0) > 0
     assert big.all()
+
+
+def test_calibration_stats_recipe():
+    s_in, s_out = inputs.calibration_stats(3, 300, 4000)
+    s_in2, s_out2 = inputs.calibration_stats(3, 300, 4000)
+    np.testing.assert_array_equal(s_in, s_in2)
+    np.testing.assert_array_equal(s_out, s_out2)
+    assert s_in.dtype == np.float32 and s_in.shape == (4000,) and s_out.shape == (300,)
+    assert np.all(s_in > 0) and np.all(s_out > 0)
+    assert abs(float(s_in.mean(dtype=np.float64)) - 1.0) < 1e-5
+    assert abs(float(s_out.mean(dtype=np.float64)) - 1.0) < 1e-5
+    # 1% of the input channels are x10 outliers: they lift the top 1% far above the
+    # log-normal tail alone (whose top 1% averages about 3.5x the median)
+    s_in3, _ = inputs.calibration_stats(3, 300, 4000, outlier_frac=0.0)
+    assert np.sort(s_in)[-40:].mean() > 6 * np.median(s_in)
+    assert np.sort(s_in3)[-40:].mean() < 6 * np.median(s_in3)
