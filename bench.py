@@ -60,7 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=400)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the GEMM / derive / CPU-baseline measurements")
-    ap.add_argument("--profile-kernel", choices=["derive", "gemv", "gemm"], default=None,
+    ap.add_argument("--profile-kernel", choices=["derive", "gemv", "gemm", "svid"], default=None,
                     help="run a few launches of one kernel (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=3, metavar=("N", "K", "M"), default=(11008, 4096, 1),
                     help="with --profile-kernel: out features, in features, batch/tokens")
@@ -778,7 +778,14 @@ def profile_kernel(args):
     L = make_layer(rabit, spec, 0, "layer", N, K, device, M)
     W = torch.from_numpy(inputs.weight(inputs.seed_for(9, 0), N, K)).to(device)
     ws = rabit.alloc_gemm_workspace(N, K, 2, M, device=device) if args.profile_kernel == "gemm" else None
-    for _ in range(args.launches):
+    if args.profile_kernel == "svid":
+        # one initialisation: T = --launches iterations, 5 power steps per update
+        s_in, s_out = inputs.calibration_stats(inputs.seed_for(9, 0), N, K)
+        sws = rabit.alloc_svid_init_workspace(N, K, 2, device=device)
+        rabit.rabit_svid_init(W, torch.from_numpy(s_in).to(device), torch.from_numpy(s_out).to(device),
+                              SVID_ALPHA_IN, SVID_ALPHA_OUT, L["a"], L["b"], L["packed"], sws, P=2,
+                              T=args.launches, power_iters=5)
+    for _ in range(args.launches if args.profile_kernel != "svid" else 0):
         if args.profile_kernel == "derive":
             rabit.rabit_derive_pack(W, L["a"], L["b"], L["packed"])
         elif args.profile_kernel == "gemv":
