@@ -434,14 +434,8 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     args.debug = debug_flags;
 
     void (*kern)(CUtensorMap, GemmArgs) = P == 2 ? gemm_kernel<2> : gemm_kernel<3>;
-    static int opted[2][64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !opted[P - 2][dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        opted[P - 2][dev] = 1;
-    }
+    static std::atomic<int> opted[2][64];
+    if (cudaError_t e = ensure_smem_optin(kern, kSmemBytes, opted[P - 2]); e != cudaSuccess) return e;
     int grid = args.num_tiles < ctx.num_sms ? args.num_tiles : ctx.num_sms;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));

@@ -848,14 +848,8 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     }
     p.pass_rows = pass_rows;
     // Opt in to the largest dynamic shared memory once per kernel and device.
-    static int opted[10][64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !opted[variant][dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
-        if (e != cudaSuccess) return e;
-        opted[variant][dev] = 1;
-    }
+    static std::atomic<int> opted[10][64];
+    if (cudaError_t e = ensure_smem_optin(kern, kSmemBudget, opted[variant]); e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(static_cast<unsigned>(threads));

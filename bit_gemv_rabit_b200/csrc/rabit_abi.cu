@@ -3,10 +3,12 @@
 // Each entry point validates every argument on the host before anything is enqueued
 // (pure argument checks first, then the device checks), then calls one launcher.  Nothing
 // here computes any part of the layer: all arithmetic runs in the CUDA kernels.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -22,11 +24,12 @@ thread_local int t_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
 struct DeviceInfo {
-    int state;  // 0 unknown, 1 ok (sm_100), 2 wrong arch
+    std::atomic<int> state;  // 0 unknown, 1 ok (sm_100), 2 wrong arch; set last, under g_devices_mutex
     int num_sms;
     uint32_t *fault_ptr;
 };
 DeviceInfo g_devices[kMaxDevices];
+std::mutex g_devices_mutex;
 
 int cuda_fail(cudaError_t e) {
     t_last_cuda_error = static_cast<int>(e);
@@ -45,23 +48,29 @@ int device_ctx(void *stream, rabit::LaunchCtx &ctx, uint32_t **fault_ptr) {
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= kMaxDevices) return RABIT_ERR_ARCH;
     DeviceInfo &info = g_devices[dev];
-    if (info.state == 0) {
-        int major = 0, minor = 0, sms = 0;
-        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
-            return cuda_fail(e);
-        if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
-            return cuda_fail(e);
-        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-            return cuda_fail(e);
-        void *fp = nullptr;
-        if (major == 10 && minor == 0) {
-            if ((e = cudaGetSymbolAddress(&fp, g_fault_word)) != cudaSuccess) return cuda_fail(e);
+    int state = info.state.load(std::memory_order_acquire);
+    if (state == 0) {
+        std::lock_guard<std::mutex> lock(g_devices_mutex);
+        state = info.state.load(std::memory_order_relaxed);
+        if (state == 0) {
+            int major = 0, minor = 0, sms = 0;
+            if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+                return cuda_fail(e);
+            if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+                return cuda_fail(e);
+            if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+                return cuda_fail(e);
+            void *fp = nullptr;
+            if (major == 10 && minor == 0) {
+                if ((e = cudaGetSymbolAddress(&fp, g_fault_word)) != cudaSuccess) return cuda_fail(e);
+            }
+            info.num_sms = sms;
+            info.fault_ptr = static_cast<uint32_t *>(fp);
+            state = (major == 10 && minor == 0) ? 1 : 2;
+            info.state.store(state, std::memory_order_release);
         }
-        info.num_sms = sms;
-        info.fault_ptr = static_cast<uint32_t *>(fp);
-        info.state = (major == 10 && minor == 0) ? 1 : 2;
     }
-    if (info.state != 1 || env_flag("RABIT_TEST_FORCE_ARCH_MISMATCH")) return RABIT_ERR_ARCH;
+    if (state != 1 || env_flag("RABIT_TEST_FORCE_ARCH_MISMATCH")) return RABIT_ERR_ARCH;
     ctx.stream = static_cast<cudaStream_t>(stream);
     ctx.num_sms = info.num_sms;
     ctx.pdl = !(std::getenv("RABIT_PDL") && std::strcmp(std::getenv("RABIT_PDL"), "0") == 0);

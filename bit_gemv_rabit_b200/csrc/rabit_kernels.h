@@ -2,11 +2,28 @@
 // Each launcher assumes its arguments were validated by the C ABI layer (rabit_abi.cu).
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 namespace rabit {
+
+// Raises `kern`'s dynamic shared-memory limit to `bytes` on the current device the first time
+// a launch there needs it.  `seen` is the kernel's per-device record; on devices past its 64
+// entries the attribute is set on every call.  Two threads making the first call at once may
+// both set it, which is harmless.
+template <typename Kern>
+inline cudaError_t ensure_smem_optin(Kern kern, int bytes, std::atomic<int> (&seen)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached && seen[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && cached) seen[dev].store(1, std::memory_order_release);
+    return e;
+}
 
 inline int64_t padded_cols(int K) { return ((static_cast<int64_t>(K) + 127) / 128) * 128; }
 

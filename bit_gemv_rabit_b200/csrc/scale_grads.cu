@@ -391,16 +391,11 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
                             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-        static int opted[2][64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
+        static std::atomic<int> opted[2][64];
         void (*kern)(CUtensorMap, const uint32_t *, const float *, const float *, int, int, int, float *, float *,
                      uint32_t *, uint64_t) = P == 2 ? scale_grads_tma_kernel<2> : scale_grads_tma_kernel<3>;
-        if (dev >= 0 && dev < 64 && !opted[P - 2][dev]) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmem);
-            if (e != cudaSuccess) return e;
-            opted[P - 2][dev] = 1;
-        }
+        e = ensure_smem_optin(kern, kTmaSmem, opted[P - 2]);
+        if (e != cudaSuccess) return e;
         nrb = (N + kBoxRows * kBoxesPerCta - 1) / (kBoxRows * kBoxesPerCta);
         cfg.gridDim = dim3(static_cast<unsigned>(nct) * static_cast<unsigned>(nrb));
         cfg.blockDim = dim3(kTmaThreads);
