@@ -749,23 +749,33 @@ def run_ours(args, rank, world, local, dist):
     if rank == 0 and world == 1 and not args.no_secondary:
         del graphs
         torch.cuda.empty_cache()
-        line["gemm"] = bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained)
-        torch.cuda.empty_cache()
-        line.update(bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained))
-        torch.cuda.empty_cache()
-        line["gemv_3path"] = bench_gemv_three_path(rabit, device, alu_peak)
-        torch.cuda.empty_cache()
-        line["scale_grads"] = bench_scale_grads(rabit, device, hbm_peak)
-        torch.cuda.empty_cache()
-        line["svid_init"] = bench_svid_init(rabit, device, hbm_peak)
-        torch.cuda.empty_cache()
-        line["decode_batch_sweep"] = bench_decode_sweep(rabit, device, alu_peak, hbm_peak)
-        torch.cuda.empty_cache()
+        secondary(line, "gemm", lambda: bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained))
+        secondary(line, "qat_step", lambda: bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained),
+                  merge=True)
+        secondary(line, "gemv_3path", lambda: bench_gemv_three_path(rabit, device, alu_peak))
+        secondary(line, "scale_grads", lambda: bench_scale_grads(rabit, device, hbm_peak))
+        secondary(line, "svid_init", lambda: bench_svid_init(rabit, device, hbm_peak))
+        secondary(line, "decode_batch_sweep", lambda: bench_decode_sweep(rabit, device, alu_peak, hbm_peak))
         prepare_oracle_inputs(base, spec)
         line["cpu_baseline"] = cpu_baseline(base, 1)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def secondary(line, key, fn, merge=False):
+    """Run one secondary measurement into the line.  A failure is recorded under `key` as an
+    error string instead of ending the run, so the headline line is always printed."""
+    try:
+        out = fn()
+        if merge:
+            line.update(out)
+        else:
+            line[key] = out
+    except Exception as exc:  # noqa: BLE001 -- any failure of a secondary figure
+        line[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    if torch.cuda.is_available():
+        torch.cuda.empty_cache()
 
 
 def profile_kernel(args):

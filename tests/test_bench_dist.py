@@ -61,3 +61,17 @@ def test_reference_arm_line_shape():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert bench.run_reference(args, 1, 2) is None
+
+
+def test_secondary_failure_is_recorded_not_raised():
+    sys.path.insert(0, ROOT)
+    import bench
+    line = {"value": 1.0}
+    bench.secondary(line, "ok", lambda: {"x": 1})
+    bench.secondary(line, "merged", lambda: {"derive_pack": {"y": 2}}, merge=True)
+
+    def boom():
+        raise RuntimeError("out of memory")
+    bench.secondary(line, "bad", boom)
+    assert line["ok"] == {"x": 1} and line["derive_pack"] == {"y": 2} and "merged" not in line
+    assert line["bad"] == {"error": "RuntimeError: out of memory"}
