@@ -10,14 +10,16 @@
  * (length K) a per-input scale (the paper's g_k and h_k).  The planes are derived in
  * sequence from one shared full-precision weight W (sec. 4.2 "The Coupled Forward Pass"):
  *     S_1 = sign(W),   R_1 = W - a_1 (.) S_1 (.) b_1,   S_2 = sign(R_1),
- * with sign(v) = +1 unless v < 0 (so +0, -0, NaN and an exact residual tie give +1).
- * Only the 2-path (2-bit) case, P = 2, is implemented.
+ * with sign(v) = +1 unless v < 0 (so +0, -0, NaN and an exact residual tie give +1), and
+ * for three paths (the 3-bit case) once more: R_2 = R_1 - a_2 (.) S_2 (.) b_2, S_3 = sign(R_2).
+ * P = 2 and P = 3 are implemented.
  *
  * Conventions shared by every call:
  *   - Every pointer argument is DEVICE memory owned by the caller (e.g. a torch tensor's
  *     data_ptr()).  The library allocates no device memory and keeps no per-call state;
- *     its only global state is a per-device fault word (rabit_read_fault) and cached
- *     device attributes.
+ *     its only global state is a per-device fault word (rabit_read_fault), cached device
+ *     attributes, and the fixed scratch buffer of rabit_gemm_noalloc (a static device
+ *     array, not an allocation).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous:
  *     they validate, enqueue and return.  Execution errors surface at the caller's next
  *     synchronisation, as for any CUDA launch.
