@@ -170,3 +170,24 @@ def test_planted_map_back_mistake_is_caught(monkeypatch):
     S1, a1, b1 = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=2, T=2)
     S2, a2, b2 = osvid.svid_init(W, 7.0 * s_in, 0.3 * s_out, ALPHA_IN, ALPHA_OUT, P=2, T=2)
     assert not np.allclose(osvid.reconstruct(S2, a2, b2), osvid.reconstruct(S1, a1, b1), rtol=1e-6)
+
+
+def test_planted_jacobi_order_is_caught_by_the_diagonal_case():
+    """Updating every path from the previous iteration's paths (instead of the paths before it
+    from this iteration, as the formula states) breaks the hand-worked diagonal case: at t = 1
+    every path would see W itself and take its largest entry."""
+    W = np.diag([3.0, -2.0, 1.0])
+    ones = np.ones(3)
+
+    def jacobi(W, P, T):
+        paths = np.zeros((P,) + W.shape)
+        for _ in range(T):
+            old = paths.copy()
+            for i in range(P):
+                S, g, h = osvid.svid(W - (old.sum(axis=0) - old[i]))
+                paths[i] = g[:, None] * S * h[None, :]
+        return paths.sum(axis=0)
+
+    assert np.linalg.norm(jacobi(W, 3, 1) - W) > 1.0
+    S, a, b = osvid.svid_init(W, ones, ones, ALPHA_IN, ALPHA_OUT, P=3, T=1)
+    assert np.linalg.norm(osvid.reconstruct(S, a, b) - W) < 1e-12
