@@ -154,3 +154,7 @@ def test_valid_arguments_without_gpu_fail_cleanly(lib):
     assert st in (CUDA, ARCH)
     flags = ctypes.c_uint32(0)
     assert lib.rabit_read_fault(None, ctypes.byref(flags), 0) in (CUDA, ARCH)
+    need = lib.rabit_svid_init_workspace_bytes(8, 16, 2)
+    st = lib.rabit_svid_init(P(FAKE), 8, 16, 16, 2, 20, 40, P(FAKE), P(FAKE), 0.8, 0.65, P(FAKE), P(FAKE),
+                             P(FAKE), P(FAKE), need, None)
+    assert st in (CUDA, ARCH)
