@@ -141,15 +141,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
                     last_parity[s] = ph;
                 }
             }
-            if (!ok) {
-                // Let every copy already in flight land before the CTA can exit.  The abort
-                // flag is raised already, so drain with a private flag that stays clear.
-                int drain_abort = 0;
-                for (int s = 0; s < kStages; ++s)
-                    if (issued[s])
-                        mbar_wait_bounded(smem_u32(&ctl->full_b[s]), last_parity[s], &drain_abort,
-                                          p.timeout_ns, p.fault, FAULT_GEMM_DRAIN);
-            }
+            // Let every copy already in flight land before the CTA can exit, also when another
+            // role stopped early on an expired wait (the abort flag may be raised, so drain with
+            // a private flag).  These are the latest phases of their stages, complete already in
+            // normal operation.
+            (void)ok;
+            int drain_abort = 0;
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s])
+                    mbar_wait_bounded(smem_u32(&ctl->full_b[s]), last_parity[s], &drain_abort,
+                                      p.timeout_ns, p.fault, FAULT_GEMM_DRAIN);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -353,20 +354,14 @@ void *tensor_map_encode_entry() {
 // device address, and that address is what the kernels receive.
 static __device__ __align__(256) uint8_t g_gemm_noalloc_scratch[RABIT_GEMM_NOALLOC_SCRATCH_BYTES];
 
-cudaError_t gemm_noalloc_scratch(void **ptr, size_t *bytes) {
-    // Looked up once per device, with that device current (the first call on each device).
-    static void *cache[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!cache[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        cache[dev] = p;
-    }
-    *ptr = cache[dev];
+cudaError_t gemm_noalloc_scratch(const LaunchCtx &ctx, void **ptr, size_t *bytes) {
+    // Looked up once per context, with the launch's device current: the symbol's address
+    // belongs to the context the module was loaded in.
+    static ContextCache<void *> cache;
+    const int st = cache.get(ctx.device, ctx.context, [](void **out) {
+        return static_cast<int>(cudaGetSymbolAddress(out, g_gemm_noalloc_scratch));
+    }, ptr);
+    if (st != 0) return static_cast<cudaError_t>(st);
     *bytes = sizeof(g_gemm_noalloc_scratch);
     return cudaSuccess;
 }
@@ -387,7 +382,26 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = ctx.pdl ? 1 : 0;
 
-    // 1. X'_k = fp16(x (.) b_k), permuted within 32-column groups.
+    // 1. Tensor map over the workspace viewed as [P][M][Kp] fp16.
+    auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap tmap;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(P)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kp) * 2, static_cast<cuuint64_t>(M) * Kp * 2};
+    cuuint32_t box[3] = {kBK, kBN, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, workspace, dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+    // 2. Shared-memory opt-in.  Steps 1 and 2 can fail, so they come before anything is
+    //    enqueued: a call that returns an error has put no work on the stream.
+    void (*kern)(CUtensorMap, GemmArgs) = P == 2 ? gemm_kernel<2> : gemm_kernel<3>;
+    static ContextFlags opted[2];
+    if (cudaError_t e = ensure_smem_optin(ctx, kern, kSmemBytes, opted[P - 2]); e != cudaSuccess) return e;
+
+    // 3. X'_k = fp16(x (.) b_k), permuted within 32-column groups.
     {
         const int64_t total = static_cast<int64_t>(P) * M * (Kp / 2);
         int64_t blocks = (total + 255) / 256;
@@ -403,20 +417,7 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
         if (e != cudaSuccess) return e;
     }
 
-    // 2. Tensor map over the workspace viewed as [P][M][Kp] fp16.
-    auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
-    if (!encode) return cudaErrorNotSupported;
-    CUtensorMap tmap;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(P)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kp) * 2, static_cast<cuuint64_t>(M) * Kp * 2};
-    cuuint32_t box[3] = {kBK, kBN, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, workspace, dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-
-    // 3. Persistent tcgen05 kernel.
+    // 4. Persistent tcgen05 kernel.
     GemmArgs args;
     args.packed = packed;
     args.a = a;
@@ -433,9 +434,6 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     args.num_tiles = args.tiles_m * tiles_n;
     args.debug = debug_flags;
 
-    void (*kern)(CUtensorMap, GemmArgs) = P == 2 ? gemm_kernel<2> : gemm_kernel<3>;
-    static std::atomic<int> opted[2][64];
-    if (cudaError_t e = ensure_smem_optin(kern, kSmemBytes, opted[P - 2]); e != cudaSuccess) return e;
     int grid = args.num_tiles < ctx.num_sms ? args.num_tiles : ctx.num_sms;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));

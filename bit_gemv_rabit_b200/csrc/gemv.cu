@@ -848,8 +848,8 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
     }
     p.pass_rows = pass_rows;
     // Opt in to the largest dynamic shared memory once per kernel and device.
-    static std::atomic<int> opted[10][64];
-    if (cudaError_t e = ensure_smem_optin(kern, kSmemBudget, opted[variant]); e != cudaSuccess) return e;
+    static ContextFlags opted[10];
+    if (cudaError_t e = ensure_smem_optin(ctx, kern, kSmemBudget, opted[variant]); e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(static_cast<unsigned>(threads));

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "rabit.h"
@@ -22,14 +23,15 @@ __device__ uint32_t g_fault_word = 0;
 
 thread_local int t_last_cuda_error = 0;
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = rabit::kCtxCacheDevices;
 struct DeviceInfo {
     std::atomic<int> state;  // 0 unknown, 1 ok (sm_100), 2 wrong arch; set last, under g_devices_mutex
     int num_sms;
-    uint32_t *fault_ptr;
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_devices_mutex;
+// Device address of g_fault_word, per device, for the context it was looked up in.
+rabit::ContextCache<uint32_t *> g_fault_ptr;
 
 int cuda_fail(cudaError_t e) {
     t_last_cuda_error = static_cast<int>(e);
@@ -39,6 +41,32 @@ int cuda_fail(cudaError_t e) {
 bool env_flag(const char *name) {
     const char *v = std::getenv(name);
     return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+// Unique id (cuCtxGetId) of the context current on the calling thread, or 0 when there is
+// none yet or the driver does not provide the calls.  The id is never reused by the driver,
+// unlike the CUcontext handle, so a context created after a reset never matches an old one.
+uint64_t current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrent get_current = [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess) ? reinterpret_cast<GetCurrent>(fn) : nullptr;
+    }();
+    static GetId get_id = [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        return (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess) ? reinterpret_cast<GetId>(fn) : nullptr;
+    }();
+    if (!get_current || !get_id) return 0;
+    CUcontext c = nullptr;
+    if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+    unsigned long long id = 0;
+    if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return static_cast<uint64_t>(id);
 }
 
 // Validates the current device; fills ctx.  Returns RABIT_OK or an error status.
@@ -60,12 +88,7 @@ int device_ctx(void *stream, rabit::LaunchCtx &ctx, uint32_t **fault_ptr) {
                 return cuda_fail(e);
             if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
                 return cuda_fail(e);
-            void *fp = nullptr;
-            if (major == 10 && minor == 0) {
-                if ((e = cudaGetSymbolAddress(&fp, g_fault_word)) != cudaSuccess) return cuda_fail(e);
-            }
             info.num_sms = sms;
-            info.fault_ptr = static_cast<uint32_t *>(fp);
             state = (major == 10 && minor == 0) ? 1 : 2;
             info.state.store(state, std::memory_order_release);
         }
@@ -74,7 +97,22 @@ int device_ctx(void *stream, rabit::LaunchCtx &ctx, uint32_t **fault_ptr) {
     ctx.stream = static_cast<cudaStream_t>(stream);
     ctx.num_sms = info.num_sms;
     ctx.pdl = !(std::getenv("RABIT_PDL") && std::strcmp(std::getenv("RABIT_PDL"), "0") == 0);
-    if (fault_ptr) *fault_ptr = info.fault_ptr;
+    ctx.device = dev;
+    ctx.context = current_context_id();
+    if (fault_ptr) {
+        // The lookup makes the device's primary context current if it was not yet, so the
+        // context id is read again afterwards for the entry and for the launch.
+        uint32_t *fp = nullptr;
+        const int st = g_fault_ptr.get(dev, ctx.context, [&](uint32_t **out) {
+            void *p = nullptr;
+            const cudaError_t err = cudaGetSymbolAddress(&p, g_fault_word);
+            *out = static_cast<uint32_t *>(p);
+            if (err == cudaSuccess) ctx.context = current_context_id();
+            return static_cast<int>(err);
+        }, &fp);
+        if (st != 0) return cuda_fail(static_cast<cudaError_t>(st));
+        *fault_ptr = fp;
+    }
     return RABIT_OK;
 }
 
@@ -123,8 +161,14 @@ int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ldw, int P, 
     return finish_launch(rabit::launch_derive_pack(ctx, W, w_dtype == RABIT_BF16, N, K, ldw, P, a, b, packed));
 }
 
+size_t rabit_gemv_workspace_bytes(int N, int K, int P, int batch) {
+    if (N < 1 || K < 1 || P < 1 || batch < 1 || batch > 16) return 0;
+    return rabit::gemv_workspace_bytes(N, K, P, batch);
+}
+
 int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
-               const void *x, int x_dtype, int batch, int ldx, float *y, int ldy, void *stream) {
+               const void *x, int x_dtype, int batch, int ldx, float *y, int ldy, void *workspace,
+               size_t workspace_bytes, void *stream) {
     if (x_dtype != RABIT_F32 && x_dtype != RABIT_BF16) return RABIT_ERR_INVALID_ARG;
     if (!packed || !a || !b || !x || !y) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || P < 1 || batch < 1 || batch > 16 || ldx < K || ldy < N)
@@ -132,12 +176,19 @@ int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, in
     if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
     if (!aligned(packed, 16)) return RABIT_ERR_ALIGNMENT;
     if (!aligned(x, x_dtype == RABIT_BF16 ? 2 : 4) || !aligned(y, 4)) return RABIT_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < rabit::gemv_workspace_bytes(N, K, P, batch)) return RABIT_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return RABIT_ERR_ALIGNMENT;
     rabit::LaunchCtx ctx;
     uint32_t *fault = nullptr;
     int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
-    return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, P, x, x_dtype == RABIT_BF16,
-                                            batch, ldx, y, ldy, fault, wait_timeout_ns()));
+    const char *which = std::getenv("RABIT_GEMV_KERNEL");
+    if (which && std::strcmp(which, "dp2a") == 0)
+        return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, P, x, x_dtype == RABIT_BF16,
+                                                batch, ldx, y, ldy, fault, wait_timeout_ns()));
+    const int debug = env_flag("RABIT_TEST_GEMV_WITHHOLD_COPY") ? 2 : 0;
+    return finish_launch(rabit::launch_gemv_tc(ctx, packed, a, b, N, K, P, x, x_dtype == RABIT_BF16, batch,
+                                               ldx, y, ldy, workspace, fault, wait_timeout_ns(), debug));
 }
 
 int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
@@ -178,7 +229,7 @@ int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, i
     if (st != RABIT_OK) return st;
     void *scratch = nullptr;
     size_t scratch_bytes = 0;
-    cudaError_t e = rabit::gemm_noalloc_scratch(&scratch, &scratch_bytes);
+    cudaError_t e = rabit::gemm_noalloc_scratch(ctx, &scratch, &scratch_bytes);
     if (e != cudaSuccess) return cuda_fail(e);
     if (need > scratch_bytes) return RABIT_ERR_WORKSPACE;
     const uint64_t timeout_ns = wait_timeout_ns();
@@ -207,8 +258,9 @@ int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed, const flo
     uint32_t *fault = nullptr;
     int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
+    const int debug = env_flag("RABIT_TEST_SCALE_GRADS_WITHHOLD_COPY") ? 1 : 0;
     return finish_launch(rabit::launch_scale_grads(ctx, G, ldg, packed, a, b, N, K, P, grad_a, grad_b,
-                                                   workspace, fault, wait_timeout_ns()));
+                                                   workspace, fault, wait_timeout_ns(), debug));
 }
 
 size_t rabit_svid_init_workspace_bytes(int N, int K, int P) {

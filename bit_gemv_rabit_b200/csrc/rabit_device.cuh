@@ -22,6 +22,7 @@ enum : uint32_t {
     FAULT_GEMM_WAIT_EPILOGUE = 1u << 3,
     FAULT_GEMM_DRAIN = 1u << 4,
     FAULT_GEMV_WAIT_COPY = 1u << 5,
+    FAULT_GEMV_WAIT_MMA = 1u << 6,
     FAULT_SCALE_GRADS_WAIT = 1u << 7,
 };
 
@@ -113,6 +114,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// L2 prefetch of one tiled box (no data reaches the SM, so it may run before the
+// programmatic-launch wait without observing a value an earlier kernel still writes).
+__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1) : "memory");
+}
+
+// Barrier over a subset of the CTA's warps (named barrier `id`, `threads` a multiple of 32).
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -142,6 +155,16 @@ __device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, 
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// D[tmem] (+)= A[tmem] x B[smem desc], kind::i8: unsigned 8-bit A, signed 8-bit B, s32
+// accumulator (exact integer arithmetic).
+__device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 __device__ __forceinline__ void tc_wait_st() {
@@ -181,6 +204,18 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)
         : "memory");
 }
 
+// Each thread of the warp reads 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored in 128-byte-swizzled
 // atoms of 8 rows x 128 bytes (1024-byte atoms stacked along the M/N dimension).
 //   bits [0,14)  start address >> 4      bits [16,30) leading-dim byte offset >> 4 (unused
@@ -201,6 +236,13 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t saddr) {
 //   bit 15/16 A/B major (0 = K)     [17,23) N >> 3              [24,29) M >> 4
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
     return (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (0u << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::i8: unsigned 8-bit A, signed 8-bit B (both K-major), s32
+// accumulator.  Same fields as above; D format 2 = s32, A format 0 = u8, B format 1 = s8.
+__host__ __device__ constexpr uint32_t idesc_u8s8_s32(int M, int N) {
+    return (2u << 4) | (0u << 7) | (1u << 10) | (0u << 15) | (0u << 16) |
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 

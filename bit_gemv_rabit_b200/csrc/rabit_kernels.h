@@ -2,38 +2,38 @@
 // Each launcher assumes its arguments were validated by the C ABI layer (rabit_abi.cu).
 #pragma once
 
-#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "ctx_cache.h"
+
 namespace rabit {
 
-// Raises `kern`'s dynamic shared-memory limit to `bytes` on the current device the first time
-// a launch there needs it.  `seen` is the kernel's per-device record; on devices past its 64
-// entries the attribute is set on every call.  Two threads making the first call at once may
-// both set it, which is harmless.
-template <typename Kern>
-inline cudaError_t ensure_smem_optin(Kern kern, int bytes, std::atomic<int> (&seen)[64]) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const bool cached = dev >= 0 && dev < 64;
-    if (cached && seen[dev].load(std::memory_order_acquire)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && cached) seen[dev].store(1, std::memory_order_release);
-    return e;
-}
-
-inline int64_t padded_cols(int K) { return ((static_cast<int64_t>(K) + 127) / 128) * 128; }
-
 // Launch configuration shared by every kernel launch: programmatic dependent launch lets a
-// kernel's prologue overlap the tail of the previous kernel on the same stream.
+// kernel's prologue overlap the tail of the previous kernel on the same stream.  `device`
+// and `context` identify where the launch goes (context = cuCtxGetId of the current
+// context, 0 if it could not be read): per-context settings are keyed on them.
 struct LaunchCtx {
     cudaStream_t stream;
     int num_sms;
     bool pdl;
+    int device;
+    uint64_t context;
 };
+
+// Raises `kern`'s dynamic shared-memory limit to `bytes` in the current context the first
+// time a launch there needs it (the attribute belongs to the context the module is loaded
+// in, so a new context after a device reset gets it again).
+template <typename Kern>
+inline cudaError_t ensure_smem_optin(const LaunchCtx &ctx, Kern kern, int bytes, ContextFlags &seen) {
+    if (seen.done(ctx.device, ctx.context)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) seen.mark(ctx.device, ctx.context);
+    return e;
+}
+
+inline int64_t padded_cols(int K) { return ((static_cast<int64_t>(K) + 127) / 128) * 128; }
 
 // P = 2 or 3 paths.
 cudaError_t launch_derive_pack(const LaunchCtx &ctx, const void *W, bool w_bf16, int N, int K,
@@ -43,13 +43,23 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
                         const float *b, int N, int K, int P, const void *x, bool x_bf16, int batch,
                         int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns);
 
+// Tensor-core decode (gemv_tc.cu).  The workspace holds one ticket per 128-row tile (must be
+// zero before the first call; every call leaves them zero) and the partial sums of the row
+// tiles shared between CTAs.
+constexpr int kGemvMaxGrid = 160;
+size_t gemv_workspace_bytes(int N, int K, int P, int batch);
+cudaError_t launch_gemv_tc(const LaunchCtx &ctx, const uint32_t *packed, const float *a, const float *b,
+                           int N, int K, int P, const void *x, bool x_bf16, int batch, int ldx, float *y,
+                           int ldy, void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug);
+
 // The driver's cuTensorMapEncodeTiled (as a PFN_cuTensorMapEncodeTiled_v12000), or null.
 void *tensor_map_encode_entry();
 
 size_t scale_grads_workspace_bytes(int N, int K, int P);
 cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, const uint32_t *packed,
                                const float *a, const float *b, int N, int K, int P, float *grad_a,
-                               float *grad_b, void *workspace, uint32_t *fault_word, uint64_t timeout_ns);
+                               float *grad_b, void *workspace, uint32_t *fault_word, uint64_t timeout_ns,
+                               int debug = 0);
 
 // Iterative Residual SVID initialisation (svid.cu).
 size_t svid_workspace_bytes(int N, int K, int P);
@@ -59,8 +69,9 @@ cudaError_t launch_svid_init(const LaunchCtx &ctx, const float *W, int ldw, int 
                              uint32_t *fault_word, uint64_t timeout_ns);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
-// Device address and size of the library's fixed GEMM scratch buffer (rabit_gemm_noalloc).
-cudaError_t gemm_noalloc_scratch(void **ptr, size_t *bytes);
+// Device address (in the launch's context) and size of the library's fixed GEMM scratch
+// buffer (rabit_gemm_noalloc).
+cudaError_t gemm_noalloc_scratch(const LaunchCtx &ctx, void **ptr, size_t *bytes);
 cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
                         const float *b, int N, int K, int P, const uint16_t *x, int M, int ldx,
                         float *y, int ldy, void *workspace, uint32_t *fault_word,

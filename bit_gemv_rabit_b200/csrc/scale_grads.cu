@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kTmaThreads)
 scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_t *__restrict__ packed,
                        const float *__restrict__ a, const float *__restrict__ b, int N, int K, int Wr,
                        float *__restrict__ ws_a, float *__restrict__ ws_b, uint32_t *fault,
-                       uint64_t timeout_ns) {
+                       uint64_t timeout_ns, int debug) {
     constexpr int kG = kP == 2 ? 2 : 4;
     constexpr int kSteps = kBoxCols / 128;
     constexpr int kRowsPerWarp = kBoxRows / 8;
@@ -210,17 +210,20 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_
                 if (!mbar_wait_bounded(smem_u32(&empty[s]), ((c / kStages) & 1) ^ 1, &abort_flag, timeout_ns,
                                        fault, FAULT_SCALE_GRADS_WAIT))
                     break;
+                if ((debug & 1) && c == 0) continue;   // fault injection: this box never comes
                 mbar_arrive_expect_tx(smem_u32(&full[s]), kBoxBytes);
                 tma_load_2d(smem_u32(stage + s * kBoxRows * kBoxCols), &tmap_g, smem_u32(&full[s]), c0,
                             row0 + c * kBoxRows);
                 issued = c + 1;
             }
-            if (abort_flag) {   // let every issued copy land before the CTA can exit
-                int drain_abort = 0;
-                for (int c = max(0, issued - kStages); c < issued; ++c)
+            // Let every issued copy land before the CTA can exit (the consumers stop early on an
+            // expired wait).  These are the latest phases of their stages, already complete in
+            // normal operation.
+            int drain_abort = 0;
+            for (int c = max(0, issued - kStages); c < issued; ++c)
+                if (!((debug & 1) && c == 0))
                     mbar_wait_bounded(smem_u32(&full[c % kStages]), (c / kStages) & 1, &drain_abort, timeout_ns,
                                       fault, FAULT_SCALE_GRADS_WAIT);
-            }
         }
         return;
     }
@@ -265,6 +268,9 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_
         const int s = c % kStages;
         const bool ok = mbar_wait_bounded(smem_u32(&full[s]), (c / kStages) & 1, &abort_flag, timeout_ns, fault,
                                           FAULT_SCALE_GRADS_WAIT);
+        // An expired wait ends this warp's boxes: it stops releasing stages, so the producer's
+        // own bounded wait expires and it drains the copies it issued before the CTA exits.
+        if (!__all_sync(0xffffffffu, ok)) break;
         const float *box = stage + s * kBoxRows * kBoxCols;
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i) {
@@ -275,8 +281,7 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_
             for (int k = 0; k < kP; ++k) racc[k] = 0.0f;
 #pragma unroll
             for (int st = 0; st < kSteps; ++st) {
-                const float4 g4 = ok ? *reinterpret_cast<const float4 *>(box + r * kBoxCols + 128 * st + 4 * lane)
-                                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                const float4 g4 = *reinterpret_cast<const float4 *>(box + r * kBoxCols + 128 * st + 4 * lane);
                 const float gvals[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
                 for (int k = 0; k < kP; ++k) {
@@ -362,7 +367,8 @@ size_t scale_grads_workspace_bytes(int N, int K, int P) {
 
 cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, const uint32_t *packed,
                                const float *a, const float *b, int N, int K, int P, float *grad_a,
-                               float *grad_b, void *workspace, uint32_t *fault_word, uint64_t timeout_ns) {
+                               float *grad_b, void *workspace, uint32_t *fault_word, uint64_t timeout_ns,
+                               int debug) {
     if (P != 2 && P != 3) return cudaErrorInvalidValue;
     const int Wr = static_cast<int>(padded_cols(K) / 32);
     const int nct = (K + tile_cols(P) - 1) / tile_cols(P);
@@ -391,16 +397,17 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
                             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-        static std::atomic<int> opted[2][64];
+        static ContextFlags opted[2];
         void (*kern)(CUtensorMap, const uint32_t *, const float *, const float *, int, int, int, float *, float *,
-                     uint32_t *, uint64_t) = P == 2 ? scale_grads_tma_kernel<2> : scale_grads_tma_kernel<3>;
-        e = ensure_smem_optin(kern, kTmaSmem, opted[P - 2]);
+                     uint32_t *, uint64_t, int) = P == 2 ? scale_grads_tma_kernel<2> : scale_grads_tma_kernel<3>;
+        e = ensure_smem_optin(ctx, kern, kTmaSmem, opted[P - 2]);
         if (e != cudaSuccess) return e;
         nrb = (N + kBoxRows * kBoxesPerCta - 1) / (kBoxRows * kBoxesPerCta);
         cfg.gridDim = dim3(static_cast<unsigned>(nct) * static_cast<unsigned>(nrb));
         cfg.blockDim = dim3(kTmaThreads);
         cfg.dynamicSmemBytes = kTmaSmem;
-        e = cudaLaunchKernelEx(&cfg, kern, tmap, packed, a, b, N, K, Wr, ws_a, ws_b, fault_word, timeout_ns);
+        e = cudaLaunchKernelEx(&cfg, kern, tmap, packed, a, b, N, K, Wr, ws_a, ws_b, fault_word, timeout_ns,
+                               debug);
     } else {
         nrb = (N + kTileRows - 1) / kTileRows;
         cfg.gridDim = dim3(static_cast<unsigned>(nct) * static_cast<unsigned>(nrb));

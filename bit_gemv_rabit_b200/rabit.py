@@ -25,7 +25,8 @@ _c, _p, _i, _sz = ctypes, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = [
     ("rabit_packed_words", _sz, [_i, _i, _i]),
     ("rabit_derive_pack", _i, [_p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
-    ("rabit_gemv", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _i, _p, _i, _p]),
+    ("rabit_gemv_workspace_bytes", _sz, [_i, _i, _i, _i]),
+    ("rabit_gemv", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_gemm_noalloc", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p]),
@@ -106,12 +107,30 @@ def rabit_derive_pack(W: torch.Tensor, a: torch.Tensor, b: torch.Tensor, packed:
     return packed
 
 
+def rabit_gemv_workspace_bytes(N: int, K: int, P: int = 2, batch: int = 1) -> int:
+    return int(load().rabit_gemv_workspace_bytes(N, K, P, batch))
+
+
+def alloc_gemv_workspace(N: int, K: int, P: int = 2, batch: int = 16, device=None) -> torch.Tensor:
+    """A zero-filled workspace for rabit_gemv (torch allocates and zero-fills it once; every
+    call leaves its counters zero, so it can be reused by later calls on the same stream)."""
+    return torch.zeros(rabit_gemv_workspace_bytes(N, K, P, batch), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
 def rabit_gemv(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,
-               x: torch.Tensor, y: torch.Tensor, P: int = 2, stream=None) -> torch.Tensor:
-    """x [batch][K] bf16/fp32 (pitch x.stride(0)); y [batch][N] fp32 out (pitch y.stride(0))."""
+               x: torch.Tensor, y: torch.Tensor, P: int = 2, workspace: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """x [batch][K] bf16/fp32 (pitch x.stride(0)); y [batch][N] fp32 out (pitch y.stride(0)).
+    workspace: from alloc_gemv_workspace (zero-filled once); when None, a fresh zero-filled one
+    is allocated for this call."""
     batch = x.shape[0]
+    if workspace is None:
+        workspace = alloc_gemv_workspace(N, K, P, batch, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
     _check(load().rabit_gemv(_dptr(packed), _dptr(a), _dptr(b), N, K, P, _dptr(x), _dtype_code(x),
-                             batch, x.stride(0), _dptr(y), y.stride(0), _stream(stream)),
+                             batch, x.stride(0), _dptr(y), y.stride(0), _dptr(workspace), ws_bytes,
+                             _stream(stream)),
            "rabit_gemv")
     return y
 

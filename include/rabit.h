@@ -25,8 +25,9 @@
  *     synchronisation, as for any CUDA launch.
  *   - Matrices are row-major; `ld*` arguments are row pitches in ELEMENTS.
  *   - Every call returns a rabit_status (0 = success).  Arguments are validated before
- *     anything is enqueued; a call that returns an error has enqueued nothing.  No call
- *     aborts, throws or prints.  RABIT_ERR_CUDA leaves the cudaError_t in
+ *     anything is enqueued; a call that returns an error has enqueued nothing, except a
+ *     RABIT_ERR_CUDA from a launch after the first of a call that enqueues several kernels
+ *     (rabit_gemm, rabit_svid_init).  No call aborts, throws or prints.  RABIT_ERR_CUDA leaves the cudaError_t in
  *     rabit_last_cuda_error() (per calling thread).
  *   - The device current on the calling thread must be an sm_100 (B200-class) GPU; any
  *     other device gives RABIT_ERR_ARCH.
@@ -101,19 +102,33 @@ RABIT_API int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ld
 /*
  * rabit_gemv -- decode path, batch 1..16 (sec. 4.1 stacking executed per path as in
  * Appendix E.1 "Compute Pipeline": paths computed in parallel, signs applied without
- * multiplication, warp-level reduction):
+ * multiplication, output scale applied last):
  *     y[beta][n] = sum_k a[k][n] * sum_j S_k[n][j] * b[k][j] * x[beta][j]
+ * The signs enter the tensor cores as their bits (u8 x s8 -> s32 products, exact); the
+ * activation term x * b_k is quantised per run of columns to 16 bits (bf16 x) or 24 bits
+ * (fp32 x) with a power-of-two scale, and results are deterministic.
  *   packed  RABIT_LAYOUT_V2 buffer of N x K, P paths (input)
  *   a [P][N], b [P][K] fp32
  *   x       [batch][ldx], bf16 (x_dtype RABIT_BF16) or fp32 (RABIT_F32), ldx >= K
  *   y       [batch][ldy] fp32 (output, fully overwritten for n < N), ldy >= N
+ *   workspace  at least rabit_gemv_workspace_bytes(N, K, P, batch) bytes, 16-byte aligned,
+ *              caller-owned (about 2.6 MB plus 4 bytes per 128 rows).  It holds the partial
+ *              sums of row tiles that several CTAs share and one counter per 128-row tile.
+ *              It MUST be zero-filled before its first use; every call leaves the counters
+ *              it used zero again, so one fill lasts for the life of the buffer, for any
+ *              shape whose size fits it.  Calls that share a workspace
+ *              must not overlap on the GPU (order them on one stream).  After a fault reported
+ *              by rabit_read_fault, zero it again.
  * Accuracy (normwise, max|y - y_exact| / max|y_exact|): <= 2e-3 for bf16 x, <= 1e-5 for
  * fp32 x.  Errors: INVALID_ARG, SHAPE (batch outside 1..16, pitches), UNSUPPORTED,
- * ALIGNMENT (packed), ARCH, CUDA.
+ * ALIGNMENT (packed, workspace), WORKSPACE, ARCH, CUDA.  A device-side wait that expires
+ * (it cannot in correct operation) ends the kernel early and is reported by
+ * rabit_read_fault as RABIT_ERR_TIMEOUT.
  */
+RABIT_API size_t rabit_gemv_workspace_bytes(int N, int K, int P, int batch);
 RABIT_API int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
                const void *x, int x_dtype, int batch, int ldx, float *y, int ldy,
-               void *stream);
+               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * rabit_gemm -- prefill / QAT forward path at large M (sec. 4.2: the forward pass uses

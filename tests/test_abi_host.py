@@ -73,9 +73,11 @@ def test_derive_pack_validation(lib):
 
 def test_gemv_validation(lib):
     f = lib.rabit_gemv
+    need = lib.rabit_gemv_workspace_bytes(8, 8, 2, 1)
     args = lambda **kw: [P(kw.get("packed", FAKE)), P(FAKE), P(FAKE), kw.get("N", 8), kw.get("K", 8),
                          kw.get("P", 2), P(kw.get("x", FAKE)), kw.get("xd", 1), kw.get("batch", 1),
-                         kw.get("ldx", 8), P(kw.get("y", FAKE)), kw.get("ldy", 8), None]
+                         kw.get("ldx", 8), P(kw.get("y", FAKE)), kw.get("ldy", 8), P(kw.get("ws", FAKE)),
+                         kw.get("wsb", need), None]
     assert f(*args(xd=5)) == INVALID
     assert f(*args(packed=0)) == INVALID
     assert f(*args(y=0)) == INVALID
@@ -88,6 +90,20 @@ def test_gemv_validation(lib):
     assert f(*args(packed=FAKE + 8)) == ALIGN
     assert f(*args(x=FAKE + 1)) == ALIGN
     assert f(*args(y=FAKE + 2)) == ALIGN
+    assert f(*args(ws=0)) == WS
+    assert f(*args(wsb=need - 1)) == WS
+    assert f(*args(ws=FAKE + 8)) == ALIGN           # workspace 16-byte alignment
+
+
+def test_gemv_workspace_size_grows_with_rows_only(lib):
+    # fixed region of partial sums, then one 4-byte counter per 128-row tile (16-byte rounded)
+    base = lib.rabit_gemv_workspace_bytes(1, 1, 2, 1)
+    assert base > 0
+    assert lib.rabit_gemv_workspace_bytes(128, 4096, 2, 16) == base
+    assert lib.rabit_gemv_workspace_bytes(4096, 4096, 3, 1) == base - 16 + 32 * 4
+    assert lib.rabit_gemv_workspace_bytes(14336, 4096, 2, 4) == base - 16 + 112 * 4
+    assert lib.rabit_gemv_workspace_bytes(8, 8, 2, 0) == 0
+    assert lib.rabit_gemv_workspace_bytes(8, 8, 2, 17) == 0
 
 
 def test_gemm_validation(lib):

@@ -1,10 +1,13 @@
 """A device wait that runs out is reported, not hung on.
 
-The GEMM's test switch RABIT_TEST_SKIP_ONE_ARRIVE makes the expansion warps skip their first
-arrival, so a bounded wait that depends on it expires (after RABIT_WAIT_TIMEOUT_MS).  The
-kernel then drains its in-flight copies, frees tensor memory and returns; the host reads
-RABIT_ERR_TIMEOUT with a GEMM wait's fault bit, and the next call on the same context is
-correct.  No GPU fault is involved: the failure is a missing arrival that a flag withholds.
+Host-side test switches withhold one event a kernel waits for:
+  - RABIT_TEST_SKIP_ONE_ARRIVE: the GEMM's expansion warps skip their first arrival;
+  - RABIT_TEST_GEMV_WITHHOLD_COPY: the decode kernel's producer never issues its first copy;
+  - RABIT_TEST_SCALE_GRADS_WITHHOLD_COPY: the scale-gradient producer never issues its first box.
+The bounded wait that depends on it expires (after RABIT_WAIT_TIMEOUT_MS); the kernel drains
+its in-flight copies, frees tensor memory and returns; the host reads RABIT_ERR_TIMEOUT with
+that wait's fault bit, and the next call on the same context is correct.  No GPU fault is
+involved: the failure is a missing event that a flag withholds.
 """
 import ctypes
 
@@ -22,6 +25,10 @@ pytestmark = pytest.mark.gpu
 # ends up waiting on the withheld arrival; whichever runs out first records its bit and the
 # others see the abort flag.
 FAULT_GEMM_WAITS = (1 << 0) | (1 << 1) | (1 << 2) | (1 << 3)
+# the decode kernel's waits: copies (producer, expansion) and the MMA issuer / epilogue /
+# expansion-group barrier; the MMA issuer starts waiting first, so its bit is usually the one
+FAULT_GEMV_WAITS = (1 << 5) | (1 << 6)
+FAULT_SCALE_GRADS_WAIT = 1 << 7
 RABIT_ERR_TIMEOUT = -8
 
 
@@ -72,3 +79,57 @@ def test_gemm_wait_expiry_is_reported_and_the_context_survives(monkeypatch):
     ref = oracle.layer(S, a, b, x)
     err = float(np.max(np.abs(y.cpu().numpy() - ref)) / np.max(np.abs(ref)))
     assert err <= 2e-3
+
+
+def _read_fault():
+    flags = ctypes.c_uint32(0)
+    st = rabit.load().rabit_read_fault(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
+                                        ctypes.byref(flags), 1)
+    return st, flags.value
+
+
+@pytest.mark.parametrize("N,K,batch", [(256, 512, 1), (4096, 4096, 4)])
+def test_gemv_copy_wait_expiry_is_reported_and_the_context_survives(monkeypatch, N, K, batch):
+    W, a, b, x, at, bt, packed, xt = _case(N, K, batch, seed=4300 + N)
+    ws = rabit.alloc_gemv_workspace(N, K, 2, batch)
+    y = torch.zeros((batch, N), device="cuda")
+    monkeypatch.setenv("RABIT_TEST_GEMV_WITHHOLD_COPY", "1")
+    monkeypatch.setenv("RABIT_WAIT_TIMEOUT_MS", "50")
+    rabit.rabit_gemv(packed, at, bt, N, K, xt, y, workspace=ws)
+    st, flags = _read_fault()
+    assert st == RABIT_ERR_TIMEOUT
+    assert flags & FAULT_GEMV_WAITS
+    monkeypatch.delenv("RABIT_TEST_GEMV_WITHHOLD_COPY")
+    monkeypatch.delenv("RABIT_WAIT_TIMEOUT_MS")
+    # after a fault the workspace is zeroed again (its tile counters may be mid-count)
+    ws.zero_()
+    rabit.rabit_gemv(packed, at, bt, N, K, xt, y, workspace=ws)
+    torch.cuda.synchronize()
+    assert rabit.rabit_read_fault(clear=True) == 0
+    ref = oracle.layer(oracle.derive_signs(W, a, b), a, b, x)
+    err = float(np.max(np.abs(y.cpu().numpy() - ref)) / np.max(np.abs(ref)))
+    assert err <= 2e-3
+
+
+def test_scale_grads_copy_wait_expiry_is_reported_and_the_context_survives(monkeypatch):
+    N, K = 512, 1024
+    W, a, b, x, at, bt, packed, xt = _case(N, K, 1, seed=4400)
+    G = torch.from_numpy(np.random.default_rng(4401).standard_normal((N, K)).astype(np.float32)).cuda()
+    ga, gb = torch.empty((2, N), device="cuda"), torch.empty((2, K), device="cuda")
+    ws = rabit.alloc_scale_grads_workspace(N, K, 2)
+    monkeypatch.setenv("RABIT_TEST_SCALE_GRADS_WITHHOLD_COPY", "1")
+    monkeypatch.setenv("RABIT_WAIT_TIMEOUT_MS", "50")
+    rabit.rabit_scale_grads(G, packed, at, bt, N, K, ga, gb, ws)
+    st, flags = _read_fault()
+    assert st == RABIT_ERR_TIMEOUT
+    assert flags & FAULT_SCALE_GRADS_WAIT
+    monkeypatch.delenv("RABIT_TEST_SCALE_GRADS_WITHHOLD_COPY")
+    monkeypatch.delenv("RABIT_WAIT_TIMEOUT_MS")
+    rabit.rabit_scale_grads(G, packed, at, bt, N, K, ga, gb, ws)
+    torch.cuda.synchronize()
+    assert rabit.rabit_read_fault(clear=True) == 0
+    S = oracle.derive_signs(W, a, b)
+    ref_a, ref_b = oracle.scale_grads(G.cpu().numpy(), S, a, b)
+    for got, ref in ((ga, ref_a), (gb, ref_b)):
+        err = float(np.max(np.abs(got.cpu().numpy() - ref)) / np.max(np.abs(ref)))
+        assert err <= 1e-5
