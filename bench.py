@@ -178,13 +178,16 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-# Sign bits the GEMV's integer dot-product pipe can apply per SM clock: dp2a issues at 64
-# lanes per clock per SM on sm_100 (measured) and each dp2a applies 2 weight bits.
-DP2A_BITS_PER_SM_CLK = 128
+# Compute bound of the decode kernel.  It feeds the sign bits to tcgen05.mma kind::i8 as one
+# byte each (the A operand, 128 rows x 32 bytes per instruction), and at M = 128 with N <= 64
+# one such instruction takes 44.8 SM clocks whatever N is (measured on this part; N = 256
+# takes 128 clocks, the full i8 rate).  So the tensor core takes in at most 4096 / 44.8 =
+# 91.4 sign bits per clock per SM, at every batch size up to 16.
+TC_SIGN_BITS_PER_SM_CLK = 91.4
 
 
-def alu_peak_gbs(device) -> tuple[float, str]:
-    """GEMV compute bound in GB/s of packed sign bits: SMs x max SM clock x 128 bits / 8."""
+def tc_peak_gbs(device) -> tuple[float, str]:
+    """Decode compute bound in GB/s of packed sign bits: SMs x max SM clock x 91.4 bits / 8."""
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     mhz = 1965.0
     try:
@@ -192,7 +195,9 @@ def alu_peak_gbs(device) -> tuple[float, str]:
             mhz = float(json.load(f).get("sm_max_mhz", mhz))
     except Exception:
         pass
-    return sms * mhz * 1e6 * DP2A_BITS_PER_SM_CLK / 8 / 1e9, f"{sms} SMs x {mhz:.0f} MHz x {DP2A_BITS_PER_SM_CLK} sign bits/clk (dp2a pipe)"
+    return (sms * mhz * 1e6 * TC_SIGN_BITS_PER_SM_CLK / 8 / 1e9,
+            f"{sms} SMs x {mhz:.0f} MHz x {TC_SIGN_BITS_PER_SM_CLK} sign bits/clk "
+            "(A-operand intake of tcgen05.mma kind::i8 at M=128, N<=64)")
 
 
 def sign_bytes(layers) -> int:
@@ -215,7 +220,8 @@ def make_layer(rabit, spec, idx, name, N, K, device, batch, P=2):
     rabit.rabit_derive_pack(torch.from_numpy(W).to(device), at, bt, packed, P=P)
     x = inputs.activations(seed, batch, K, channel_outlier_frac=spec["x_outliers"])
     return dict(name=name, N=N, K=K, P=P, a=at, b=bt, packed=packed, x_host=x,
-                x=bf16_tensor(x, device), y=torch.empty((batch, N), device=device))
+                x=bf16_tensor(x, device), y=torch.empty((batch, N), device=device),
+                ws=rabit.alloc_gemv_workspace(N, K, P, min(batch, 16), device=device) if batch <= 16 else None)
 
 
 def decode_bytes(layers, batch=1):
@@ -302,15 +308,44 @@ def bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained):
     ms = timed_replays(graphs, steps, 5, None, device)
     flops = sum(2 * 2 * M * L["N"] * L["K"] for L in sets[0])
     tflops = flops * steps / (ms * 1e-3) / 1e12
+    fp8 = measure_fp8_tflops(device)
+    roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
+            "frac": round(tflops / tf_peak, 4),
+            "peak_note": "measured dense bf16 burst; fp16 operands have the same nominal rate",
+            "frac_of_nominal_fp8_dense_4500": round(tflops / 4500.0, 4)}
+    if fp8 is not None:
+        roof["fp8_dense_measured_tflops"] = fp8
+        roof["frac_of_measured_fp8_dense"] = round(tflops / fp8, 4)
     return {"workload": "llama3_8b_mlp_prefill_m2048", "value": round(tflops, 1), "unit": "TFLOP/s",
             "dtype": "fp16", "ms_per_step": round(ms / steps, 4), "launches_per_step": 2 * len(sets[0]),
-            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_peak,
-                         "unit": "TFLOP/s", "frac": round(tflops / tf_peak, 4),
-                         "peak_note": "measured dense bf16 burst; fp16 operands have the same nominal rate",
-                         "frac_of_nominal_fp8_dense_4500": round(tflops / 4500.0, 4)}}
+            "roofline": roof}
 
 
-def bench_decode_sweep(rabit, device, alu_peak, hbm_peak):
+def measure_fp8_tflops(device, n=8192, reps=10):
+    """Dense e4m3 GEMM throughput of this part (torch._scaled_mm, n^3, best of reps): the
+    denominator for an fp8 fraction.  None when the call is not available."""
+    try:
+        a = torch.randn((n, n), device=device).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=device).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=device)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 1)
+    except Exception:
+        return None
+
+
+def bench_decode_sweep(rabit, device, tc_peak, hbm_peak):
     """Llama-3-8B-shaped decode set (q 4096x4096, k/v 1024x4096, gate/up 14336x4096, down
     4096x14336, 0.1% x20 weight outliers) at batch 1, 4, 8 and 16: microseconds per set and per
     layer, three rotated copies of the packed weights (more than L2)."""
@@ -326,7 +361,8 @@ def bench_decode_sweep(rabit, device, alu_peak, hbm_peak):
         def step_fn(layers, B=B):
             def f():
                 for L in layers:
-                    rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"][:B], L["y"][:B])
+                    rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"][:B], L["y"][:B],
+                                     workspace=L["ws"])
             return f
 
         graphs = [capture_graph(step_fn(ls)) for ls in sets]
@@ -338,8 +374,8 @@ def bench_decode_sweep(rabit, device, alu_peak, hbm_peak):
             "us_per_set": round(us, 2), "us_per_layer": round(us / len(base), 2),
             "GB_per_s": round(byts / (us * 1e-6) / 1e9, 1),
             "hbm_frac": round(byts / (us * 1e-6) / 1e9 / hbm_peak, 4),
-            # the dp2a pipe applies B sign bits per weight bit at batch B
-            "alu_frac": round(B * sign / (us * 1e-6) / 1e9 / alu_peak, 4)}
+            # the tensor core takes each sign bit in once for all B batch rows (N <= 64)
+            "tensor_frac": round(sign / (us * 1e-6) / 1e9 / tc_peak, 4)}
         del graphs
     del sets, base
     torch.cuda.empty_cache()
@@ -356,12 +392,13 @@ def warm_launch_us(rabit, layers, device):
         if key in out:
             continue
         g = capture_graph(lambda L=L: [rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"],
-                                                        L["x"], L["y"], P=L["P"]) for _ in range(200)])
+                                                        L["x"], L["y"], P=L["P"], workspace=L["ws"])
+                                       for _ in range(200)])
         out[key] = round(timed_replays([g], 5, 2, None, device) / 5 / 200 * 1e3, 2)
     return out
 
 
-def bench_gemv_three_path(rabit, device, alu_peak):
+def bench_gemv_three_path(rabit, device, tc_peak, hbm_peak):
     """The 3-bit variant (three paths) on the same Llama-2-7B decode set, batch 1, ten rotated
     copies (the pages' Table 7 reports 3-bit kernel latencies beside the 2-bit ones)."""
     spec = inputs.WORKLOADS[WORKLOAD]
@@ -373,7 +410,8 @@ def bench_gemv_three_path(rabit, device, alu_peak):
     def step_fn(layers):
         def f():
             for L in layers:
-                rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"], P=3)
+                rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"], P=3,
+                                 workspace=L["ws"])
         return f
 
     graphs = [capture_graph(step_fn(ls)) for ls in sets]
@@ -385,9 +423,12 @@ def bench_gemv_three_path(rabit, device, alu_peak):
     return {"workload": "llama2_7b_decode_b1_3path", "value": round(algo * steps / (ms * 1e-3) / 1e9, 1),
             "unit": "GB/s", "us_per_set": round(ms / steps * 1e3, 2),
             "us_per_launch_warm_l2_by_shape": warm_launch_us(rabit, base, device),
-            "roofline": {"bound": "alu", "achieved": round(sign * steps / (ms * 1e-3) / 1e9, 1),
-                         "peak": round(alu_peak, 1), "unit": "GB/s",
-                         "frac": round(sign * steps / (ms * 1e-3) / 1e9 / alu_peak, 4)},
+            "roofline": {"bound": "hbm", "achieved": round(algo * steps / (ms * 1e-3) / 1e9, 1),
+                         "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(algo * steps / (ms * 1e-3) / 1e9 / hbm_peak, 4)},
+            "roofline_compute": {"bound": "tensor", "achieved": round(sign * steps / (ms * 1e-3) / 1e9, 1),
+                                 "peak": round(tc_peak, 1), "unit": "GB/s",
+                                 "frac": round(sign * steps / (ms * 1e-3) / 1e9 / tc_peak, 4)},
             "note": "3 sign words + 1 padding word per group in HBM; algorithmic bytes count the 3 signs"}
 
 
@@ -680,8 +721,10 @@ def run_ours(args, rank, world, local, dist):
     launches = len(base) * args.steps
     per_launch_us = elapsed_ms * 1e3 / launches
     achieved = step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
-    alu_peak, alu_kind = alu_peak_gbs(device)
-    alu_achieved = sign_bytes(base) * args.steps / (elapsed_ms * 1e-3) / 1e9
+    tc_peak, tc_kind = tc_peak_gbs(device)
+    tc_achieved = sign_bytes(base) * args.steps / (elapsed_ms * 1e-3) / 1e9
+    # every bounded device wait of the timed region must have completed
+    fault = rabit.rabit_read_fault(clear=True)
 
     # ---- end to end through the public API: pinned host x in, y back to the host, per step
     e2e_steps = min(args.e2e_steps, args.steps)
@@ -695,7 +738,7 @@ def run_ours(args, rank, world, local, dist):
         layers = sets[s % COPIES]
         for L, xp, yp in zip(layers, x_pinned, y_pinned):
             L["x"].copy_(xp, non_blocking=True)
-            rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"])
+            rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"], workspace=L["ws"])
             yp.copy_(L["y"], non_blocking=True)
         stream.synchronize()
 
@@ -710,6 +753,7 @@ def run_ours(args, rank, world, local, dist):
     torch.cuda.synchronize()
     e2e_ms, e2e_units = aggregate(e0.elapsed_time(e1), float(step_bytes) * e2e_steps, dist, device)
     e2e_value = e2e_units / (e2e_ms * 1e-3) / 1e9
+    fault |= rabit.rabit_read_fault(clear=True)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -723,17 +767,19 @@ def run_ours(args, rank, world, local, dist):
                          f"({COPIES * step_bytes / 1e6:.0f} MB) rotated per step",
                    "launch": "CUDA graph per copy, programmatic dependent launch between kernels",
                    "parallelism": f"replica x{world}"},
-        # The GEMV is bound by its integer dot-product pipe before HBM (DP2A_BITS_PER_SM_CLK):
-        # the roofline is that pipe; the HBM fraction (the metric's "% of peak") is beside it.
-        "roofline": {"bound": "alu", "achieved": round(alu_achieved, 2), "peak": round(alu_peak, 1),
-                     "unit": "GB/s", "frac": round(alu_achieved / alu_peak, 4), "traffic": None,
-                     "kernel": "gemv_kernel", "avg_launch_us": round(per_launch_us, 3),
-                     "peak_kind": alu_kind, "achieved_kind": "packed sign bytes per second"},
-        "roofline_hbm": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(achieved / hbm_peak, 4),
-                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                         "achieved_kind": "algorithmic bytes (signs, scales, x, y) per second"},
+        # The metric's "% of peak": algorithmic bytes of the decode pass over the measured HBM
+        # copy bandwidth.  The tensor core's intake of sign bits (TC_SIGN_BITS_PER_SM_CLK) is the
+        # compute bound beside it.
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                     "kernel": "gemv_tc_kernel", "avg_launch_us": round(per_launch_us, 3),
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "achieved_kind": "algorithmic bytes (signs, scales, x, y) per launch / average launch time"},
+        "roofline_compute": {"bound": "tensor", "achieved": round(tc_achieved, 2), "peak": round(tc_peak, 1),
+                             "unit": "GB/s", "frac": round(tc_achieved / tc_peak, 4), "peak_kind": tc_kind,
+                             "achieved_kind": "packed sign bytes per second"},
         "gpu_launches": launches,
+        "fault_word": fault,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "api": "bit_gemv_rabit_b200.rabit.rabit_gemv per matrix, pinned host copies, stream sync per step"},
@@ -752,15 +798,36 @@ def run_ours(args, rank, world, local, dist):
         secondary(line, "gemm", lambda: bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained))
         secondary(line, "qat_step", lambda: bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained),
                   merge=True)
-        secondary(line, "gemv_3path", lambda: bench_gemv_three_path(rabit, device, alu_peak))
+        secondary(line, "gemv_3path", lambda: bench_gemv_three_path(rabit, device, tc_peak, hbm_peak))
         secondary(line, "scale_grads", lambda: bench_scale_grads(rabit, device, hbm_peak))
         secondary(line, "svid_init", lambda: bench_svid_init(rabit, device, hbm_peak))
-        secondary(line, "decode_batch_sweep", lambda: bench_decode_sweep(rabit, device, alu_peak, hbm_peak))
+        secondary(line, "decode_batch_sweep", lambda: bench_decode_sweep(rabit, device, tc_peak, hbm_peak))
+    if rank == 0:
+        # parity of the timed configuration: every output of the last timed step against the
+        # float64 oracle (normwise, per matrix; the bar is 2e-3 for bf16 activations)
         prepare_oracle_inputs(base, spec)
-        line["cpu_baseline"] = cpu_baseline(base, 1)
+        line["parity"] = timed_parity(base)
+        if world == 1 and not args.no_secondary:
+            line["cpu_baseline"] = cpu_baseline(base, 1)
+        line["fault_word"] |= rabit.rabit_read_fault(clear=True)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if line["fault_word"] or not line.get("parity", {}).get("ok", True):
+        return 1   # a bounded device wait expired, or the timed outputs are out of tolerance
     return 0
+
+
+def timed_parity(layers, tol=2e-3):
+    """Normwise error of each layer's y (from the last timed step) against the oracle."""
+    import oracle
+    errs = {}
+    for L in layers:
+        ref = oracle.layer(L["S_cache"], L["a_host"], L["b_host"], L["x_host"])
+        y = L["y"].cpu().numpy().astype(np.float64)
+        errs[L["name"]] = float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-300))
+    worst = max(errs.values())
+    return {"normwise_max": worst, "tol": tol, "ok": worst <= tol, "vs": "float64 oracle",
+            "outputs": "every row of the 7 layers, last timed step", "by_matrix": errs}
 
 
 def secondary(line, key, fn, merge=False):
@@ -799,7 +866,7 @@ def profile_kernel(args):
         if args.profile_kernel == "derive":
             rabit.rabit_derive_pack(W, L["a"], L["b"], L["packed"])
         elif args.profile_kernel == "gemv":
-            rabit.rabit_gemv(L["packed"], L["a"], L["b"], N, K, L["x"], L["y"])
+            rabit.rabit_gemv(L["packed"], L["a"], L["b"], N, K, L["x"], L["y"], workspace=L["ws"])
         else:
             rabit.rabit_gemm(L["packed"], L["a"], L["b"], N, K, L["x"], L["y"], ws)
     torch.cuda.synchronize()
@@ -809,21 +876,28 @@ def profile_kernel(args):
 
 
 def _load_traffic():
-    """DRAM bytes per GEMV launch of this workload from the committed ncu summary, or None
-    when there is none or the GEMV source changed since the counters were taken."""
+    """DRAM bytes per decode launch of this workload from the committed ncu summary, or None
+    when there is none or the kernel source changed since the counters were taken (the hash
+    covers the kernel's own file and the device helpers it includes)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "gemv_traffic.json")
-    src = os.path.join(ROOT, "bit_gemv_rabit_b200", "csrc", "gemv.cu")
     try:
         with open(path) as f:
             d = json.load(f)
-        with open(src, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-        if d.get("gemv_cu_sha256") != digest:
+        if d.get("kernel_sha256") != kernel_source_sha256():
             return None
         return d.get("bytes_per_launch")
     except Exception:
         return None
+
+
+def kernel_source_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ("gemv_tc.cu", "rabit_device.cuh"):
+        with open(os.path.join(ROOT, "bit_gemv_rabit_b200", "csrc", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 if __name__ == "__main__":
