@@ -166,6 +166,19 @@ size_t rabit_gemv_workspace_bytes(int N, int K, int P, int batch) {
     return rabit::gemv_workspace_bytes(N, K, P, batch);
 }
 
+namespace {
+// Checks one layer of a decode call (rabit_gemv, rabit_gemv_grouped); RABIT_OK or an error.
+int check_gemv_layer(const rabit_gemv_layer &l, int P, int x_dtype, int batch) {
+    if (!l.packed || !l.a || !l.b || !l.x || !l.y) return RABIT_ERR_INVALID_ARG;
+    if (l.N < 1 || l.K < 1 || l.ldx < l.K || l.ldy < l.N) return RABIT_ERR_SHAPE;
+    if (!aligned(l.packed, 16)) return RABIT_ERR_ALIGNMENT;
+    if (!aligned(l.x, x_dtype == RABIT_BF16 ? 2 : 4) || !aligned(l.y, 4)) return RABIT_ERR_ALIGNMENT;
+    (void)P;
+    (void)batch;
+    return RABIT_OK;
+}
+}  // namespace
+
 int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,
                const void *x, int x_dtype, int batch, int ldx, float *y, int ldy, void *workspace,
                size_t workspace_bytes, void *stream) {
@@ -189,6 +202,41 @@ int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, in
     const int debug = env_flag("RABIT_TEST_GEMV_WITHHOLD_COPY") ? 2 : 0;
     return finish_launch(rabit::launch_gemv_tc(ctx, packed, a, b, N, K, P, x, x_dtype == RABIT_BF16, batch,
                                                ldx, y, ldy, workspace, fault, wait_timeout_ns(), debug));
+}
+
+size_t rabit_gemv_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count) {
+    if (!layers || count < 1 || count > RABIT_GEMV_MAX_GROUP) return 0;
+    rabit::GemvLayer g[RABIT_GEMV_MAX_GROUP];
+    for (int i = 0; i < count; ++i) {
+        if (layers[i].N < 1) return 0;
+        g[i] = rabit::GemvLayer{layers[i].packed, layers[i].a, layers[i].b, layers[i].N, layers[i].K,
+                                layers[i].x, layers[i].ldx, layers[i].y, layers[i].ldy};
+    }
+    return rabit::gemv_group_workspace_bytes(g, count);
+}
+
+int rabit_gemv_grouped(const rabit_gemv_layer *layers, int count, int P, int x_dtype, int batch,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (x_dtype != RABIT_F32 && x_dtype != RABIT_BF16) return RABIT_ERR_INVALID_ARG;
+    if (!layers || count < 1 || count > RABIT_GEMV_MAX_GROUP) return RABIT_ERR_INVALID_ARG;
+    if (P < 1 || batch < 1 || batch > 16) return RABIT_ERR_SHAPE;
+    rabit::GemvLayer g[RABIT_GEMV_MAX_GROUP];
+    for (int i = 0; i < count; ++i) {
+        const int st = check_gemv_layer(layers[i], P, x_dtype, batch);
+        if (st != RABIT_OK) return st;
+        g[i] = rabit::GemvLayer{layers[i].packed, layers[i].a, layers[i].b, layers[i].N, layers[i].K,
+                                layers[i].x, layers[i].ldx, layers[i].y, layers[i].ldy};
+    }
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < rabit::gemv_group_workspace_bytes(g, count)) return RABIT_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
+    if (st != RABIT_OK) return st;
+    const int debug = env_flag("RABIT_TEST_GEMV_WITHHOLD_COPY") ? 2 : 0;
+    return finish_launch(rabit::launch_gemv_group(ctx, g, count, P, x_dtype == RABIT_BF16, batch, workspace, fault,
+                                                  wait_timeout_ns(), debug));
 }
 
 int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,

@@ -47,7 +47,20 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
 // zero before the first call; every call leaves them zero) and the partial sums of the row
 // tiles shared between CTAs.
 constexpr int kGemvMaxGrid = 160;
+constexpr int kGemvMaxGroup = 8;   // layers one grouped launch may take
+struct GemvLayer {
+    const uint32_t *packed;
+    const float *a, *b;
+    int N, K;
+    const void *x;
+    int ldx;
+    float *y;
+    int ldy;
+};
 size_t gemv_workspace_bytes(int N, int K, int P, int batch);
+size_t gemv_group_workspace_bytes(const GemvLayer *layers, int count);
+cudaError_t launch_gemv_group(const LaunchCtx &ctx, const GemvLayer *layers, int count, int P, bool x_bf16,
+                              int batch, void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug);
 cudaError_t launch_gemv_tc(const LaunchCtx &ctx, const uint32_t *packed, const float *a, const float *b,
                            int N, int K, int P, const void *x, bool x_bf16, int batch, int ldx, float *y,
                            int ldy, void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug);

@@ -27,6 +27,8 @@ SIGNATURES = [
     ("rabit_derive_pack", _i, [_p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     ("rabit_gemv_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemv", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _i, _p, _i, _p, _sz, _p]),
+    ("rabit_gemv_grouped_workspace_bytes", _sz, [_p, _i]),
+    ("rabit_gemv_grouped", _i, [_p, _i, _i, _i, _i, _p, _sz, _p]),
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_gemm_noalloc", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p]),
@@ -133,6 +135,45 @@ def rabit_gemv(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K
                              _stream(stream)),
            "rabit_gemv")
     return y
+
+
+class GemvLayer(ctypes.Structure):
+    """struct rabit_gemv_layer of include/rabit.h."""
+    _fields_ = [("packed", ctypes.c_void_p), ("a", ctypes.c_void_p), ("b", ctypes.c_void_p),
+                ("N", ctypes.c_int), ("K", ctypes.c_int), ("x", ctypes.c_void_p), ("ldx", ctypes.c_int),
+                ("y", ctypes.c_void_p), ("ldy", ctypes.c_int)]
+
+
+def _layer_array(layers):
+    arr = (GemvLayer * len(layers))()
+    for i, (packed, a, b, N, K, x, y) in enumerate(layers):
+        arr[i] = GemvLayer(packed.data_ptr(), a.data_ptr(), b.data_ptr(), N, K, x.data_ptr(), x.stride(0),
+                           y.data_ptr(), y.stride(0))
+    return arr
+
+
+def rabit_gemv_grouped_workspace_bytes(layers) -> int:
+    """layers: sequence of (packed, a, b, N, K, x, y) tuples."""
+    arr = _layer_array(layers)
+    return int(load().rabit_gemv_grouped_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers)))
+
+
+def alloc_gemv_grouped_workspace(layers, device=None) -> torch.Tensor:
+    return torch.zeros(rabit_gemv_grouped_workspace_bytes(layers), dtype=torch.uint8, device=device or "cuda")
+
+
+def rabit_gemv_grouped(layers, P: int = 2, workspace: torch.Tensor | None = None, stream=None):
+    """layers: sequence of (packed, a, b, N, K, x, y); every x has the same batch and dtype.
+    One launch computes rabit_gemv for each layer."""
+    arr = _layer_array(layers)
+    x0 = layers[0][5]
+    if workspace is None:
+        workspace = alloc_gemv_grouped_workspace(layers, device=x0.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().rabit_gemv_grouped(ctypes.cast(arr, ctypes.c_void_p), len(layers), P, _dtype_code(x0),
+                                     x0.shape[0], _dptr(workspace), ws_bytes, _stream(stream)),
+           "rabit_gemv_grouped")
+    return [layer[6] for layer in layers]
 
 
 def rabit_gemm(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,

@@ -131,6 +131,35 @@ RABIT_API int rabit_gemv(const uint32_t *packed, const float *a, const float *b,
                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * rabit_gemv_grouped -- rabit_gemv for up to RABIT_GEMV_MAX_GROUP independent layers in one
+ * launch, e.g. the projections of a decoder block that read the same activation (query, key
+ * and value; gate and up).  Each layer computes exactly what rabit_gemv computes for it; the
+ * launch shares the fixed costs (setup, the dependency on the previous kernel, the final
+ * sums) and balances all layers' work over the SMs.  The layers share P, the activation type
+ * and the batch; each has its own signs, scales, x and y (which must not overlap another
+ * layer's y).
+ *   layers     host array of `count` descriptions (1 <= count <= RABIT_GEMV_MAX_GROUP); the
+ *              pointers inside are device pointers with the layouts of rabit_gemv
+ *   workspace  at least rabit_gemv_grouped_workspace_bytes(layers, count) bytes, with the
+ *              rules of rabit_gemv's workspace (zero-filled before first use)
+ * Errors: as rabit_gemv, plus INVALID_ARG for a null `layers` or count out of range.
+ */
+#define RABIT_GEMV_MAX_GROUP 8
+typedef struct rabit_gemv_layer {
+    const uint32_t *packed;   /* RABIT_LAYOUT_V2 signs of N x K, P paths */
+    const float *a;           /* [P][N] */
+    const float *b;           /* [P][K] */
+    int N, K;
+    const void *x;            /* [batch][ldx] */
+    int ldx;
+    float *y;                 /* [batch][ldy] */
+    int ldy;
+} rabit_gemv_layer;
+RABIT_API size_t rabit_gemv_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count);
+RABIT_API int rabit_gemv_grouped(const rabit_gemv_layer *layers, int count, int P, int x_dtype, int batch,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * rabit_gemm -- prefill / QAT forward path at large M (sec. 4.2: the forward pass uses
  * W_hat^(2)), the same contraction as rabit_gemv for M tokens:
  *     y[m][n] = sum_k a[k][n] * sum_j S_k[n][j] * b[k][j] * x[m][j]

@@ -174,3 +174,27 @@ def test_valid_arguments_without_gpu_fail_cleanly(lib):
     st = lib.rabit_svid_init(P(FAKE), 8, 16, 16, 2, 20, 40, P(FAKE), P(FAKE), 0.8, 0.65, P(FAKE), P(FAKE),
                              P(FAKE), P(FAKE), need, None)
     assert st in (CUDA, ARCH)
+
+
+def test_gemv_grouped_validation(lib):
+    L = rabit.GemvLayer
+    good = dict(packed=FAKE, a=FAKE, b=FAKE, N=8, K=8, x=FAKE, ldx=8, y=FAKE, ldy=8)
+    def arr(**kw):
+        d = dict(good, **kw)
+        a = (L * 2)(L(**good), L(**d))
+        return ctypes.cast(a, ctypes.c_void_p)
+    need = lib.rabit_gemv_grouped_workspace_bytes(arr(), 2)
+    assert need == lib.rabit_gemv_workspace_bytes(16, 8, 2, 1)    # two one-tile layers
+    f = lib.rabit_gemv_grouped
+    assert f(None, 2, 2, 1, 1, P(FAKE), need, None) == INVALID
+    assert f(arr(), 0, 2, 1, 1, P(FAKE), need, None) == INVALID
+    assert f(arr(), 9, 2, 1, 1, P(FAKE), need, None) == INVALID
+    assert f(arr(), 2, 2, 7, 1, P(FAKE), need, None) == INVALID       # dtype
+    assert f(arr(), 2, 2, 1, 17, P(FAKE), need, None) == SHAPE        # batch
+    assert f(arr(y=0), 2, 2, 1, 1, P(FAKE), need, None) == INVALID
+    assert f(arr(K=0), 2, 2, 1, 1, P(FAKE), need, None) == SHAPE
+    assert f(arr(ldy=7), 2, 2, 1, 1, P(FAKE), need, None) == SHAPE
+    assert f(arr(packed=FAKE + 4), 2, 2, 1, 1, P(FAKE), need, None) == ALIGN
+    assert f(arr(), 2, 4, 1, 1, P(FAKE), need, None) == UNSUP
+    assert f(arr(), 2, 2, 1, 1, P(FAKE), need - 1, None) == WS
+    assert f(arr(), 2, 2, 1, 1, P(FAKE + 8), need, None) == ALIGN
