@@ -204,15 +204,18 @@ int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, in
                                                ldx, y, ldy, workspace, fault, wait_timeout_ns(), debug));
 }
 
-size_t rabit_gemv_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count) {
+size_t rabit_gemv_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count, int P, int x_dtype,
+                                          int batch) {
     if (!layers || count < 1 || count > RABIT_GEMV_MAX_GROUP) return 0;
+    if ((P != 2 && P != 3) || batch < 1 || batch > 16) return 0;
+    if (x_dtype != RABIT_F32 && x_dtype != RABIT_BF16) return 0;
     rabit::GemvLayer g[RABIT_GEMV_MAX_GROUP];
     for (int i = 0; i < count; ++i) {
-        if (layers[i].N < 1) return 0;
+        if (layers[i].N < 1 || layers[i].K < 1) return 0;
         g[i] = rabit::GemvLayer{layers[i].packed, layers[i].a, layers[i].b, layers[i].N, layers[i].K,
                                 layers[i].x, layers[i].ldx, layers[i].y, layers[i].ldy};
     }
-    return rabit::gemv_group_workspace_bytes(g, count);
+    return rabit::gemv_group_workspace_bytes(g, count, P, x_dtype == RABIT_BF16, batch);
 }
 
 int rabit_gemv_grouped(const rabit_gemv_layer *layers, int count, int P, int x_dtype, int batch,
@@ -228,7 +231,8 @@ int rabit_gemv_grouped(const rabit_gemv_layer *layers, int count, int P, int x_d
                                 layers[i].x, layers[i].ldx, layers[i].y, layers[i].ldy};
     }
     if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
-    if (!workspace || workspace_bytes < rabit::gemv_group_workspace_bytes(g, count)) return RABIT_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < rabit::gemv_group_workspace_bytes(g, count, P, x_dtype == RABIT_BF16, batch))
+        return RABIT_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return RABIT_ERR_ALIGNMENT;
     rabit::LaunchCtx ctx;
     uint32_t *fault = nullptr;

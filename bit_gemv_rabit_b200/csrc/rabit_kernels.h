@@ -43,9 +43,10 @@ cudaError_t launch_gemv(const LaunchCtx &ctx, const uint32_t *packed, const floa
                         const float *b, int N, int K, int P, const void *x, bool x_bf16, int batch,
                         int ldx, float *y, int ldy, uint32_t *fault_word, uint64_t timeout_ns);
 
-// Tensor-core decode (gemv_tc.cu).  The workspace holds one ticket per 128-row tile (must be
-// zero before the first call; every call leaves them zero) and the partial sums of the row
-// tiles shared between CTAs.
+// Tensor-core decode (gemv_tc.cu): a prep kernel (row scales, the B operand images, the
+// fix-up counters) and the main kernel.  The workspace holds the partial sums of the row tiles
+// shared between CTAs, one counter per 128-row tile, the row scales and the B images; every
+// call rewrites what it uses, so it needs no initialisation.
 constexpr int kGemvMaxGrid = 160;
 constexpr int kGemvMaxGroup = 8;   // layers one grouped launch may take
 struct GemvLayer {
@@ -57,8 +58,9 @@ struct GemvLayer {
     float *y;
     int ldy;
 };
+// Enough for either activation type.
 size_t gemv_workspace_bytes(int N, int K, int P, int batch);
-size_t gemv_group_workspace_bytes(const GemvLayer *layers, int count);
+size_t gemv_group_workspace_bytes(const GemvLayer *layers, int count, int P, bool x_bf16, int batch);
 cudaError_t launch_gemv_group(const LaunchCtx &ctx, const GemvLayer *layers, int count, int P, bool x_bf16,
                               int batch, void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug);
 cudaError_t launch_gemv_tc(const LaunchCtx &ctx, const uint32_t *packed, const float *a, const float *b,

@@ -27,7 +27,7 @@ SIGNATURES = [
     ("rabit_derive_pack", _i, [_p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     ("rabit_gemv_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemv", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _i, _p, _i, _p, _sz, _p]),
-    ("rabit_gemv_grouped_workspace_bytes", _sz, [_p, _i]),
+    ("rabit_gemv_grouped_workspace_bytes", _sz, [_p, _i, _i, _i, _i]),
     ("rabit_gemv_grouped", _i, [_p, _i, _i, _i, _i, _p, _sz, _p]),
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
@@ -114,8 +114,8 @@ def rabit_gemv_workspace_bytes(N: int, K: int, P: int = 2, batch: int = 1) -> in
 
 
 def alloc_gemv_workspace(N: int, K: int, P: int = 2, batch: int = 16, device=None) -> torch.Tensor:
-    """A zero-filled workspace for rabit_gemv (torch allocates and zero-fills it once; every
-    call leaves its counters zero, so it can be reused by later calls on the same stream)."""
+    """A workspace for rabit_gemv, large enough for batch rows of either x type; reusable by
+    later calls on the same stream (every call writes what it reads)."""
     return torch.zeros(rabit_gemv_workspace_bytes(N, K, P, batch), dtype=torch.uint8,
                        device=device or "cuda")
 
@@ -124,8 +124,8 @@ def rabit_gemv(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K
                x: torch.Tensor, y: torch.Tensor, P: int = 2, workspace: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """x [batch][K] bf16/fp32 (pitch x.stride(0)); y [batch][N] fp32 out (pitch y.stride(0)).
-    workspace: from alloc_gemv_workspace (zero-filled once); when None, a fresh zero-filled one
-    is allocated for this call."""
+    workspace: from alloc_gemv_workspace (needs no initialisation); when None, a fresh one is
+    allocated for this call."""
     batch = x.shape[0]
     if workspace is None:
         workspace = alloc_gemv_workspace(N, K, P, batch, device=x.device)
@@ -152,14 +152,17 @@ def _layer_array(layers):
     return arr
 
 
-def rabit_gemv_grouped_workspace_bytes(layers) -> int:
-    """layers: sequence of (packed, a, b, N, K, x, y) tuples."""
+def rabit_gemv_grouped_workspace_bytes(layers, P: int = 2) -> int:
+    """layers: sequence of (packed, a, b, N, K, x, y) tuples; every x has the same batch and
+    dtype."""
     arr = _layer_array(layers)
-    return int(load().rabit_gemv_grouped_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers)))
+    x0 = layers[0][5]
+    return int(load().rabit_gemv_grouped_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers), P,
+                                                         _dtype_code(x0), x0.shape[0]))
 
 
-def alloc_gemv_grouped_workspace(layers, device=None) -> torch.Tensor:
-    return torch.zeros(rabit_gemv_grouped_workspace_bytes(layers), dtype=torch.uint8, device=device or "cuda")
+def alloc_gemv_grouped_workspace(layers, P: int = 2, device=None) -> torch.Tensor:
+    return torch.empty(rabit_gemv_grouped_workspace_bytes(layers, P), dtype=torch.uint8, device=device or "cuda")
 
 
 def rabit_gemv_grouped(layers, P: int = 2, workspace: torch.Tensor | None = None, stream=None):
@@ -168,7 +171,7 @@ def rabit_gemv_grouped(layers, P: int = 2, workspace: torch.Tensor | None = None
     arr = _layer_array(layers)
     x0 = layers[0][5]
     if workspace is None:
-        workspace = alloc_gemv_grouped_workspace(layers, device=x0.device)
+        workspace = alloc_gemv_grouped_workspace(layers, P, device=x0.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(load().rabit_gemv_grouped(ctypes.cast(arr, ctypes.c_void_p), len(layers), P, _dtype_code(x0),
                                      x0.shape[0], _dptr(workspace), ws_bytes, _stream(stream)),

@@ -104,21 +104,22 @@ RABIT_API int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ld
  * Appendix E.1 "Compute Pipeline": paths computed in parallel, signs applied without
  * multiplication, output scale applied last):
  *     y[beta][n] = sum_k a[k][n] * sum_j S_k[n][j] * b[k][j] * x[beta][j]
- * The signs enter the tensor cores as their bits (u8 x s8 -> s32 products, exact); the
- * activation term x * b_k is quantised per run of columns to 16 bits (bf16 x) or 24 bits
- * (fp32 x) with a power-of-two scale, and results are deterministic.
+ * The signs enter the tensor cores as 4-bit +-1 values and the activation term
+ * z = b_k * x (an fp32 product) as balanced base-4 digits of zq = rint(z * 2^e): one
+ * power-of-two scale per (path, batch row) puts |zq| below 2^15 (bf16 x) or 2^23 (fp32 x).
+ * The sign sums of zq are exact; results are deterministic.  Two kernels run on `stream`:
+ * one prepares the digits and scales in the workspace, the other streams the signs.
  *   packed  RABIT_LAYOUT_V2 buffer of N x K, P paths (input)
  *   a [P][N], b [P][K] fp32
  *   x       [batch][ldx], bf16 (x_dtype RABIT_BF16) or fp32 (RABIT_F32), ldx >= K
  *   y       [batch][ldy] fp32 (output, fully overwritten for n < N), ldy >= N
- *   workspace  at least rabit_gemv_workspace_bytes(N, K, P, batch) bytes, 16-byte aligned,
- *              caller-owned (about 2.6 MB plus 4 bytes per 128 rows).  It holds the partial
- *              sums of row tiles that several CTAs share and one counter per 128-row tile.
- *              It MUST be zero-filled before its first use; every call leaves the counters
- *              it used zero again, so one fill lasts for the life of the buffer, for any
- *              shape whose size fits it.  Calls that share a workspace
- *              must not overlap on the GPU (order them on one stream).  After a fault reported
- *              by rabit_read_fault, zero it again.
+ *   workspace  at least rabit_gemv_workspace_bytes(N, K, P, batch) bytes (enough for either
+ *              x type), 16-byte aligned, caller-owned: about 5.2 MB of partial sums for the
+ *              row tiles that several CTAs share, one counter per 128-row tile, the scales,
+ *              and the digits (P * K * batch bytes for bf16 x, 1.5 times that for fp32 x,
+ *              rounded up).  It needs no initialisation: every call writes what it reads.
+ *              Calls that share a workspace must not overlap on the GPU (order them on one
+ *              stream).
  * Accuracy (normwise, max|y - y_exact| / max|y_exact|): <= 2e-3 for bf16 x, <= 1e-5 for
  * fp32 x.  Errors: INVALID_ARG, SHAPE (batch outside 1..16, pitches), UNSUPPORTED,
  * ALIGNMENT (packed, workspace), WORKSPACE, ARCH, CUDA.  A device-side wait that expires
@@ -140,8 +141,9 @@ RABIT_API int rabit_gemv(const uint32_t *packed, const float *a, const float *b,
  * layer's y).
  *   layers     host array of `count` descriptions (1 <= count <= RABIT_GEMV_MAX_GROUP); the
  *              pointers inside are device pointers with the layouts of rabit_gemv
- *   workspace  at least rabit_gemv_grouped_workspace_bytes(layers, count) bytes, with the
- *              rules of rabit_gemv's workspace (zero-filled before first use)
+ *   workspace  at least rabit_gemv_grouped_workspace_bytes(layers, count, P, x_dtype, batch)
+ *              bytes, 16-byte aligned, with the rules of rabit_gemv's workspace (0 from the
+ *              size call means invalid arguments)
  * Errors: as rabit_gemv, plus INVALID_ARG for a null `layers` or count out of range.
  */
 #define RABIT_GEMV_MAX_GROUP 8
@@ -155,7 +157,8 @@ typedef struct rabit_gemv_layer {
     float *y;                 /* [batch][ldy] */
     int ldy;
 } rabit_gemv_layer;
-RABIT_API size_t rabit_gemv_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count);
+RABIT_API size_t rabit_gemv_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count, int P,
+                                                    int x_dtype, int batch);
 RABIT_API int rabit_gemv_grouped(const rabit_gemv_layer *layers, int count, int P, int x_dtype, int batch,
                                  void *workspace, size_t workspace_bytes, void *stream);
 

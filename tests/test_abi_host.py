@@ -95,13 +95,20 @@ def test_gemv_validation(lib):
     assert f(*args(ws=FAKE + 8)) == ALIGN           # workspace 16-byte alignment
 
 
-def test_gemv_workspace_size_grows_with_rows_only(lib):
-    # fixed region of partial sums, then one 4-byte counter per 128-row tile (16-byte rounded)
-    base = lib.rabit_gemv_workspace_bytes(1, 1, 2, 1)
-    assert base > 0
-    assert lib.rabit_gemv_workspace_bytes(128, 4096, 2, 16) == base
-    assert lib.rabit_gemv_workspace_bytes(4096, 4096, 3, 1) == base - 16 + 32 * 4
-    assert lib.rabit_gemv_workspace_bytes(14336, 4096, 2, 4) == base - 16 + 112 * 4
+PARTIAL_BYTES = 160 * 2 * 16 * 256 * 4     # partial sums: largest grid x 2 tiles x 16 rows x 256
+
+
+def test_gemv_workspace_layout(lib):
+    # partial sums, then the counters (4 bytes per 128-row tile) and the scales (4 bytes per
+    # path and batch row), each rounded up to 1 KiB, then the digit images: per 256 columns
+    # and path, 128 bytes per digit row (12 per batch row for fp32 x, rounded up to 8 rows)
+    assert lib.rabit_gemv_workspace_bytes(4096, 4096, 2, 1) == PARTIAL_BYTES + 1024 + 1024 + 16 * 2 * 16 * 128
+    assert lib.rabit_gemv_workspace_bytes(300, 1000, 3, 3) == PARTIAL_BYTES + 1024 + 1024 + 4 * 3 * 40 * 128
+    for N, K, P, batch in [(1, 1, 2, 1), (14336, 4096, 2, 4), (4096, 11008, 2, 16), (4096, 4096, 3, 16)]:
+        w = lib.rabit_gemv_workspace_bytes(N, K, P, batch)
+        pairs = -(-K // 256)
+        assert w >= PARTIAL_BYTES + 4 * -(-N // 128) + 4 * P * batch + pairs * P * 128 * 12 * batch
+        assert w <= PARTIAL_BYTES + 4 * -(-N // 128) + 2048 + 4 * P * batch + pairs * P * 128 * 24 * batch
     assert lib.rabit_gemv_workspace_bytes(8, 8, 2, 0) == 0
     assert lib.rabit_gemv_workspace_bytes(8, 8, 2, 17) == 0
 
@@ -183,8 +190,12 @@ def test_gemv_grouped_validation(lib):
         d = dict(good, **kw)
         a = (L * 2)(L(**good), L(**d))
         return ctypes.cast(a, ctypes.c_void_p)
-    need = lib.rabit_gemv_grouped_workspace_bytes(arr(), 2)
-    assert need == lib.rabit_gemv_workspace_bytes(16, 8, 2, 1)    # two one-tile layers
+    need = lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 2, 1, 1)
+    # two one-tile, one-unit layers, bf16 x, batch 1: 8 digit rows of 128 bytes per path
+    assert need == PARTIAL_BYTES + 1024 + 1024 + 2 * 2 * 8 * 128
+    assert lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 4, 1, 1) == 0
+    assert lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 2, 7, 1) == 0
+    assert lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 2, 1, 17) == 0
     f = lib.rabit_gemv_grouped
     assert f(None, 2, 2, 1, 1, P(FAKE), need, None) == INVALID
     assert f(arr(), 0, 2, 1, 1, P(FAKE), need, None) == INVALID
