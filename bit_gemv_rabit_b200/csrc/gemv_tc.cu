@@ -26,11 +26,12 @@
 //   fp32, and t = sum_s 4^s D_s is formed exactly in 64-bit integers.  The only roundings are
 //   z itself, its quantisation and the conversion of t to fp32.
 //
-// Two kernels per call:
-//   gemv_prep_kernel  one CTA per (layer, batch row, 2048 columns): the row's maximum |z| per
-//                     path, its scale, and the B operand of its columns for every path, written
-//                     to the workspace as the exact shared-memory image the tensor core reads,
-//                     so the main kernel moves it with one bulk copy per unit.  It also clears
+// Three kernels per call, chained by programmatic dependent launch:
+//   gemv_blockmax_kernel, gemv_prep_kernel  one CTA per (layer, batch row, 1024 columns): the
+//                     maximum |z| of the block per path, then the row's scale from the block
+//                     maxima and the B operand of the block for every path, written to the
+//                     workspace as the exact shared-memory image the tensor core reads (the main
+//                     kernel moves it with bulk copies of about 32 KiB).  The first also clears
 //                     the fix-up counters.
 //   gemv_tc_kernel    the signs.  A unit is one 128-byte-wide TMA box of packed words: 128 or
 //                     256 rows (one or two halves; a row tile has the same height) x 512
@@ -44,21 +45,22 @@
 //                     leave fp32 partial sums in the workspace, and the last contributor to
 //                     arrive (a counter per tile) adds them in contributor order, which is the
 //                     column order, so results are deterministic.
-// Roles of gemv_tc_kernel (15 warps; each group of four covers the four tensor-memory lane
+// Roles of gemv_tc_kernel (25 warps; each group of four covers the four tensor-memory lane
 // quarters):
 //   warp 0        producer: per unit one TMA box of packed sign words into a ring of stages,
 //                 and per run of units about 32 KiB of B images at a time (one bulk copy) into
 //                 a second ring.  The boxes of the first pass over the ring are requested
 //                 before the programmatic-launch wait (the kernel this one waits for, the prep
 //                 kernel, does not write the signs); the B images after it.
-//   warps 1, 14   MMA issuers (warp 1 also owns the tensor memory): one lane each issues the
-//                 MMAs of its share of the paths (M = 128, N = rows of B, K = 64; four per
-//                 256-column pair, half and path) into the run's accumulators.
+//   warps 1, 22..24  MMA issuers (warp 1 also owns the tensor memory): one lane each issues
+//                 the MMAs of one half and path (M = 128, N = rows of B, K = 64; four per
+//                 256-column pair) into the run's accumulators.  One issuing thread sustains
+//                 about one MMA per 50 clocks, far below the tensor core, hence four.
 //   warps 2..5    epilogue: per run, t from the accumulators, scaled by 2^-e and a, then the
 //                 output or the partial and the fix-up.
-//   warps 6..13   expansion: the sign words of a unit from shared memory into A stages in
-//                 tensor memory (one per half and pair); with two halves warps 6..9 take the
-//                 first half and 10..13 the second, with one half they take even and odd units.
+//   warps 6..21   expansion: the sign words of a unit from shared memory into A stages in
+//                 tensor memory, one stage per (half, 256-column pair); four groups of four
+//                 warps, group g filling stage g, so four stages are expanded at once.
 // Every wait on another agent is bounded; an expired wait records a fault bit, and the CTA
 // drains what it has in flight and exits.
 #include <cuda.h>
@@ -81,11 +83,13 @@ constexpr int kSfCols = 32;             // tensor-memory columns holding the (co
 constexpr int kMaxWStages = 8;
 constexpr int kMaxAStages = 4;
 constexpr int kMaxBBufs = 2;
-constexpr int kPrefetchUnits = 8;       // boxes a CTA prefetches to L2 beyond its first ring
+constexpr int kPrefetchUnits = 0;       // boxes a CTA prefetches to L2 before the wait (they would
+                                        // delay the prep kernel's reads, which gate the MMAs)
 constexpr int kEarlyBoxes = 2;          // boxes requested before the programmatic-launch wait
-constexpr int kThreads = 15 * 32;
-constexpr int kWarpIssuer1 = 14;        // the second MMA issuer
-constexpr int kPrepThreads = 256;
+constexpr int kThreads = 25 * 32;
+constexpr int kWarpExpand0 = 6;         // expansion warps 6..21: four groups of four
+constexpr int kWarpIssuer1 = 22;        // MMA issuers 1..3 are warps 22..24
+constexpr int kPrepThreads = 128;      // small enough to share an SM with a main-kernel CTA
 constexpr int kPrepCols = 8 * kPrepThreads;   // columns per prep CTA
 
 template <int kP> struct Geometry {
@@ -115,10 +119,23 @@ struct PrepArgs {
     PrepLayer layer[kGemvMaxGroup];
     uint8_t *img;           // [slices][layers][pairs][P][nm rows x 128 bytes]
     float *inv;             // [layer][P][batch]: 2^-e
+    float *bmax;            // [layer][P][batch][maxblk]: max |z| of each block of columns
     int *tickets;           // fix-up counters of the main kernel, cleared here
     long long slice_bytes;
-    int ntickets, nprob, batch, slice, nm;
+    int ntickets, nprob, batch, slice, nm, maxblk;
 };
+
+// The (layer, batch row, column block) of a prep CTA.
+__device__ __forceinline__ void prep_coords(const PrepArgs &p, int &l, int &beta, int &blk) {
+    int bid = blockIdx.x;
+    l = 0;
+    while (l + 1 < p.nprob && bid >= p.layer[l].blocks * p.batch) {
+        bid -= p.layer[l].blocks * p.batch;
+        ++l;
+    }
+    beta = bid / p.layer[l].blocks;
+    blk = bid - beta * p.layer[l].blocks;
+}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -201,69 +218,60 @@ __device__ __forceinline__ float load_x(const void *xrow, int j) {
     else return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(xrow)[j]) << 16);
 }
 
+// First prep kernel: the max |z| of each path over the block's 1024 columns (8 per thread),
+// one value per (layer, path, batch row, block).  It also clears the fix-up counters.
 template <bool kF32X, int kP>
 __global__ void __launch_bounds__(kPrepThreads)
-gemv_prep_kernel(const __grid_constant__ PrepArgs p) {
-    using Dg = Digits<kF32X>;
-    constexpr int kD = Dg::kD;
+gemv_blockmax_kernel(const __grid_constant__ PrepArgs p) {
     __shared__ float red[kP][kPrepThreads / 32];
-    // x and b may come from the previous kernel on the stream.  The main kernel of this call
-    // may start once every CTA is past this point: it reads nothing of ours before its own wait.
+    // x and b may come from the previous kernel on the stream; the next kernel of this call
+    // reads what we write only after its own wait.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (blockIdx.x == 0)
         for (int i = tid; i < p.ntickets; i += kPrepThreads) p.tickets[i] = 0;
-    int bid = blockIdx.x, l = 0;
-    while (l + 1 < p.nprob && bid >= p.layer[l].blocks * p.batch) {
-        bid -= p.layer[l].blocks * p.batch;
-        ++l;
-    }
+    int l, beta, blk;
+    prep_coords(p, l, beta, blk);
     const PrepLayer &q = p.layer[l];
-    const int beta = bid / q.blocks, blk = bid - beta * q.blocks;
     const int K = q.K;
     const float *b = q.b;
     const void *xrow = static_cast<const uint8_t *>(q.x) +
                        static_cast<int64_t>(beta) * q.ldx * (kF32X ? 4 : 2);
-
-    // ---- the row's max |z| per path; every CTA of the row reads the whole row (from L2)
     float mx[kP];
 #pragma unroll
     for (int k = 0; k < kP; ++k) mx[k] = 0.0f;
-    int j0 = 0;
-    if (q.vec) {
-        const int n8 = K / 8;
-        for (int i = tid; i < n8; i += kPrepThreads) {
-            float xv[8];
-            if constexpr (kF32X) {
-                const float4 v0 = reinterpret_cast<const float4 *>(xrow)[2 * i];
-                const float4 v1 = reinterpret_cast<const float4 *>(xrow)[2 * i + 1];
-                xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
-                xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
-            } else {
-                const uint4 v = reinterpret_cast<const uint4 *>(xrow)[i];
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const int c0 = blk * kPrepCols + 8 * tid;
+    if (q.vec && c0 + 8 <= K) {
+        float xv[8];
+        if constexpr (kF32X) {
+            const float4 v0 = reinterpret_cast<const float4 *>(xrow)[c0 / 4];
+            const float4 v1 = reinterpret_cast<const float4 *>(xrow)[c0 / 4 + 1];
+            xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
+            xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
+        } else {
+            const uint4 v = reinterpret_cast<const uint4 *>(xrow)[c0 / 8];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    xv[2 * h] = __uint_as_float(w[h] << 16);
-                    xv[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < kP; ++k) {
-                const float4 b0 = reinterpret_cast<const float4 *>(b + static_cast<int64_t>(k) * K)[2 * i];
-                const float4 b1 = reinterpret_cast<const float4 *>(b + static_cast<int64_t>(k) * K)[2 * i + 1];
-                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                for (int h = 0; h < 8; ++h) mx[k] = fmaxf(mx[k], fabsf(__fmul_rn(bv[h], xv[h])));
+            for (int h = 0; h < 4; ++h) {
+                xv[2 * h] = __uint_as_float(w[h] << 16);
+                xv[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
             }
         }
-        j0 = n8 * 8;
-    }
-    for (int j = j0 + tid; j < K; j += kPrepThreads) {
-        const float xv = load_x<kF32X>(xrow, j);
 #pragma unroll
-        for (int k = 0; k < kP; ++k) mx[k] = fmaxf(mx[k], fabsf(__fmul_rn(b[static_cast<int64_t>(k) * K + j], xv)));
+        for (int k = 0; k < kP; ++k) {
+            const float4 b0 = reinterpret_cast<const float4 *>(b + static_cast<int64_t>(k) * K)[c0 / 4];
+            const float4 b1 = reinterpret_cast<const float4 *>(b + static_cast<int64_t>(k) * K)[c0 / 4 + 1];
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int h = 0; h < 8; ++h) mx[k] = fmaxf(mx[k], fabsf(__fmul_rn(bv[h], xv[h])));
+        }
+    } else {
+        for (int c = c0; c < min(c0 + 8, K); ++c) {
+            const float xv = load_x<kF32X>(xrow, c);
+#pragma unroll
+            for (int k = 0; k < kP; ++k) mx[k] = fmaxf(mx[k], fabsf(__fmul_rn(b[static_cast<int64_t>(k) * K + c], xv)));
+        }
     }
 #pragma unroll
     for (int k = 0; k < kP; ++k) {
@@ -271,12 +279,38 @@ gemv_prep_kernel(const __grid_constant__ PrepArgs p) {
         if (lane == 0) red[k][warp] = mx[k];
     }
     __syncthreads();
+    if (tid < kP) {
+        float m = red[tid][0];
+#pragma unroll
+        for (int w = 1; w < kPrepThreads / 32; ++w) m = fmaxf(m, red[tid][w]);
+        p.bmax[((static_cast<int64_t>(l) * kP + tid) * p.batch + beta) * p.maxblk + blk] = m;
+    }
+}
+
+// Second prep kernel: the row's scale from the block maxima, then the B images of the block.
+template <bool kF32X, int kP>
+__global__ void __launch_bounds__(kPrepThreads)
+gemv_prep_kernel(const __grid_constant__ PrepArgs p) {
+    using Dg = Digits<kF32X>;
+    constexpr int kD = Dg::kD;
+    // The block maxima come from the previous kernel.  The main kernel of this call may start
+    // once every CTA is past this point: it reads nothing of ours before its own wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int tid = threadIdx.x;
+    int l, beta, blk;
+    prep_coords(p, l, beta, blk);
+    const PrepLayer &q = p.layer[l];
+    const int K = q.K;
+    const float *b = q.b;
+    const void *xrow = static_cast<const uint8_t *>(q.x) +
+                       static_cast<int64_t>(beta) * q.ldx * (kF32X ? 4 : 2);
     float sc[kP];
 #pragma unroll
     for (int k = 0; k < kP; ++k) {
-        float m = red[k][0];
-#pragma unroll
-        for (int w = 1; w < kPrepThreads / 32; ++w) m = fmaxf(m, red[k][w]);
+        const float *bm = p.bmax + ((static_cast<int64_t>(l) * kP + k) * p.batch + beta) * p.maxblk;
+        float m = 0.0f;
+        for (int i = 0; i < q.blocks; ++i) m = fmaxf(m, bm[i]);
         const int e = row_exponent(m, Dg::kTop, Dg::kZqLimit);
         sc[k] = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
         if (blk == 0 && tid == k)
@@ -375,7 +409,7 @@ struct Ctl {
     uint64_t a_empty[kMaxAStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
-    uint64_t drain[2];                 // one per MMA issuer
+    uint64_t drain[4];                 // one per MMA issuer
     uint64_t group;                    // barrier of the epilogue warps (bounded, unlike bar.sync)
     uint32_t tmem_base;
     int abort;
@@ -493,14 +527,10 @@ __device__ __forceinline__ bool warp_wait_idle(uint32_t bar, uint32_t parity, co
 }
 
 // A stage j of the tensor-memory ring holds the signs of (unit i, half h, pair q) with
-// j = (i * mh + h) * kUpp + q.  The expansion group that fills it: the half h (two halves),
-// else the pair q (one half, two pairs per unit), else the unit's parity.
+// j = (i * mh + h) * kUpp + q, in stage j % n_a, which expansion group j % n_a fills.
 template <int kUpp>
 __device__ __forceinline__ uint32_t a_seq(int i, int h, int q, int mh) {
     return static_cast<uint32_t>((i * mh + h) * kUpp + q);
-}
-__host__ __device__ inline int a_group(int i, int h, int q, int mh, int upp) {
-    return mh == 2 ? h : (upp == 2 ? q : i % 2);
 }
 
 template <bool kF32X, int kP>
@@ -521,7 +551,8 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
     const long long u0 = range_begin(U, G, cta), u1 = range_begin(U, G, cta + 1);
     const int mh = p.mh;
     const int tile_rows = kRows * mh;
-    const int n_issuers = mh;                       // one per half
+    // MMA issuers: two per half, one for path 0 (and path 2 when there are three), one for path 1
+    const int n_issuers = 2 * mh;
     const uint32_t pair_bytes = static_cast<uint32_t>(kP * p.nm * 128);
     volatile int *abort_flag = &ctl->abort;
     // Tensor memory: scale factors (all 1.0) at [0, 32); accumulator of set s, half h, path k
@@ -532,8 +563,8 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.n_w; ++s) {
             mbar_init(smem_u32(&ctl->w_full[s]), 1);
-            // the expansion warps that read it: both groups unless they take alternate units
-            mbar_init(smem_u32(&ctl->w_empty[s]), (mh == 2 || kUpp == 2) ? 8 : 4);
+            // the expansion warps that read it: four per group with a triple in the unit
+            mbar_init(smem_u32(&ctl->w_empty[s]), 4 * std::min(p.n_a, mh * kUpp));
         }
         for (int s = 0; s < p.n_b; ++s) {
             mbar_init(smem_u32(&ctl->b_full[s]), 1);
@@ -541,13 +572,13 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
         }
         for (int s = 0; s < p.n_a; ++s) {
             mbar_init(smem_u32(&ctl->a_full[s]), 4);
-            mbar_init(smem_u32(&ctl->a_empty[s]), 1);       // the issuer that reads it
+            mbar_init(smem_u32(&ctl->a_empty[s]), 2);       // the two issuers of its half
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&ctl->acc_full[s]), n_issuers);
             mbar_init(smem_u32(&ctl->acc_empty[s]), 4);
-            mbar_init(smem_u32(&ctl->drain[s]), 1);
         }
+        for (int s = 0; s < 4; ++s) mbar_init(smem_u32(&ctl->drain[s]), 1);
         mbar_init(smem_u32(&ctl->group), 4);
         ctl->abort = 0;
         ctl->last = 0;
@@ -670,11 +701,12 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
                     mbar_wait_bounded(smem_u32(&ctl->b_full[s]), blast_parity[s], &drain_abort, p.timeout_ns,
                                       p.fault, FAULT_GEMM_DRAIN);
         }
-    } else if (warp == 1 || warp == kWarpIssuer1) {
+    } else if (warp == 1 || warp >= kWarpIssuer1) {
         // ------------------------------------------------------------ MMA issuers
-        // One per half: issuer h issues every MMA of half h (all pairs and paths) from the A
-        // stages expansion group h fills, so each wait and commit covers 4 * kP MMAs.
-        const int issuer = warp == 1 ? 0 : 1;
+        // Issuer ii issues the MMAs of half ii / 2 for path ii % 2 (and path 2 with issuer 0 of the
+        // half): one issuing thread sustains only about one MMA per 50 clocks, so the MMAs are
+        // spread over four threads.
+        const int issuer = warp == 1 ? 0 : warp - kWarpIssuer1 + 1;
         if (lane == 0 && issuer < n_issuers) {
             const uint32_t idesc = idesc_mxf4_f32(kRows, p.nm);
             // Descriptors are built once; per MMA only their start fields move (the start
@@ -684,7 +716,7 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
             const uint32_t pair16 = pair_bytes >> 4;
             const uint32_t path16 = static_cast<uint32_t>(p.nm * 128) >> 4;
             const uint32_t set_cols = static_cast<uint32_t>(mh * kP * p.acc_stride);
-            const int h = issuer;
+            const int h = issuer >> 1, kfirst = issuer & 1;
             int bb = 0, i = 0;
             uint32_t bpar = 0, run = 0;
             bool ok = true, any = false;
@@ -727,7 +759,7 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
                             const uint32_t a0 = tmem + a_col0 + slot * static_cast<uint32_t>(kP * 32);
                             const uint32_t acc = (v != 0 || qq != 0) ? 1u : 0u;
 #pragma unroll
-                            for (int k = 0; k < kP; ++k) {
+                            for (int k = kfirst; k < kP; k += 2) {
                                 const uint32_t dk = dh + static_cast<uint32_t>(k * p.acc_stride);
                                 const uint32_t ak = a0 + static_cast<uint32_t>(k * 32);
                                 const uint64_t bk = bp + static_cast<uint64_t>(static_cast<uint32_t>(k) * path16);
@@ -760,63 +792,70 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
                                   FAULT_GEMM_DRAIN);
             }
         }
-    } else if (warp >= 6) {
+    } else if (warp >= kWarpExpand0 && warp < kWarpIssuer1) {
         // ------------------------------------------------------------ expansion of the sign words
-        const int grp = (warp - 6) >> 2;
+        // Group g (warps 6 + 4g .. 9 + 4g, one per lane quarter) fills A stage g: the signs of
+        // the (unit, half, pair) triples whose sequence index j is g modulo the stage count.
+        const int grp = (warp - kWarpExpand0) >> 2;
         const int q4 = warp & 3;                     // lane quarter this warp may access
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-        const bool by_parity = mh == 1 && kUpp == 1; // groups take alternate units
-        const int h = mh == 2 ? grp : 0;
-        const int q_lo = (mh == 1 && kUpp == 2) ? grp : 0;
-        const int q_hi = (mh == 1 && kUpp == 2) ? grp + 1 : kUpp;
-        const int brow = h * kRows + q4 * 32 + lane; // row inside the box
         const int n_units = static_cast<int>(u1 - u0);
-        for (int i = by_parity ? grp : 0; i < n_units; i += by_parity ? 2 : 1) {
-            const int st = i % p.n_w;
-            if (!warp_wait(smem_u32(&ctl->w_full[st]), static_cast<uint32_t>(i / p.n_w) & 1u, p, ctl,
-                           FAULT_GEMV_WAIT_COPY))
-                break;
-            // 128-byte box rows, swizzled in 16-byte chunks (chunk c of row r at c ^ (r % 8)),
-            // so a warp's 16-byte reads hit every bank once.
-            const uint8_t *src = wring + st * p.w_bytes + brow * 128;
-            uint32_t wd[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * (c ^ (brow & 7)));
-                wd[4 * c] = v.x; wd[4 * c + 1] = v.y; wd[4 * c + 2] = v.z; wd[4 * c + 3] = v.w;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl->w_empty[st]));
-            bool ok = true;
-#pragma unroll
-            for (int qq = 0; qq < kUpp; ++qq) {
-                if (qq < q_lo || qq >= q_hi) continue;
-                const uint32_t j = a_seq<kUpp>(i, h, qq, mh);
-                const uint32_t slot = j % static_cast<uint32_t>(p.n_a);
-                if (!warp_wait(smem_u32(&ctl->a_empty[slot]), ((j / p.n_a) & 1u) ^ 1u, p, ctl, FAULT_GEMV_WAIT_MMA)) {
-                    ok = false;
+        if (grp < p.n_a) {
+            const uint32_t slot = static_cast<uint32_t>(grp);
+            for (int i = 0; i < n_units; ++i) {
+                // does this group take a triple of unit i?  (j runs over i * mh * kUpp + 0 ..)
+                const uint32_t jb = a_seq<kUpp>(i, 0, 0, mh);
+                const uint32_t nper = static_cast<uint32_t>(mh * kUpp);
+                const uint32_t first = (slot + static_cast<uint32_t>(p.n_a) - jb % static_cast<uint32_t>(p.n_a)) %
+                                       static_cast<uint32_t>(p.n_a);
+                if (first >= nper) continue;
+                const int st = i % p.n_w;
+                if (!warp_wait(smem_u32(&ctl->w_full[st]), static_cast<uint32_t>(i / p.n_w) & 1u, p, ctl,
+                               FAULT_GEMV_WAIT_COPY))
                     break;
-                }
-                tc_fence_after();
+                bool ok = true;
+                for (uint32_t o = first; o < nper; o += static_cast<uint32_t>(p.n_a)) {
+                    const uint32_t j = jb + o;
+                    const int h = static_cast<int>(o) / kUpp, qq = static_cast<int>(o) % kUpp;
+                    // 128-byte box rows, swizzled in 16-byte chunks (chunk c of row r at c ^ (r % 8)),
+                    // so a warp's 16-byte reads hit every bank once.  Pair qq of the row is chunks
+                    // [4 qq, 4 qq + 4) with two paths, the whole row with three.
+                    const int brow = h * kRows + q4 * 32 + lane;
+                    const uint8_t *src = wring + st * p.w_bytes + brow * 128;
+                    constexpr int kChunks = 8 / kUpp;
+                    uint32_t wd[4 * kChunks];
 #pragma unroll
-                for (int k = 0; k < kP; ++k) {
-                    uint32_t v[32];
-#pragma unroll
-                    for (int g = 0; g < kUnitGroups; ++g) {
-                        const uint32_t w = wd[(qq * kUnitGroups + g) * Geometry<kP>::kGroupWords + k];
-                        v[4 * g + 0] = ((w << 3) & 0x88888888u) | 0x22222222u;
-                        v[4 * g + 1] = ((w << 2) & 0x88888888u) | 0x22222222u;
-                        v[4 * g + 2] = ((w << 1) & 0x88888888u) | 0x22222222u;
-                        v[4 * g + 3] = (w & 0x88888888u) | 0x22222222u;
+                    for (int c = 0; c < kChunks; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * ((qq * kChunks + c) ^ (brow & 7)));
+                        wd[4 * c] = v.x; wd[4 * c + 1] = v.y; wd[4 * c + 2] = v.z; wd[4 * c + 3] = v.w;
                     }
-                    tmem_st_32x32b_x32(tmem + lane_addr + a_col0 + (slot * kP + k) * 32u, v);
+                    if (!warp_wait(smem_u32(&ctl->a_empty[slot]), ((j / p.n_a) & 1u) ^ 1u, p, ctl, FAULT_GEMV_WAIT_MMA)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kP; ++k) {
+                        uint32_t v[32];
+#pragma unroll
+                        for (int g = 0; g < kUnitGroups; ++g) {
+                            const uint32_t w = wd[g * Geometry<kP>::kGroupWords + k];
+                            v[4 * g + 0] = ((w << 3) & 0x88888888u) | 0x22222222u;
+                            v[4 * g + 1] = ((w << 2) & 0x88888888u) | 0x22222222u;
+                            v[4 * g + 2] = ((w << 1) & 0x88888888u) | 0x22222222u;
+                            v[4 * g + 3] = (w & 0x88888888u) | 0x22222222u;
+                        }
+                        tmem_st_32x32b_x32(tmem + lane_addr + a_col0 + (slot * kP + k) * 32u, v);
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&ctl->a_full[slot]));
                 }
-                tc_wait_st();
-                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl->a_full[slot]));
+                if (lane == 0) mbar_arrive(smem_u32(&ctl->w_empty[st]));   // this warp is done with the box
+                if (!ok) break;
             }
-            if (!ok) break;
         }
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..5)
@@ -918,10 +957,13 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
                     for (int beta = 0; beta < kMaxBatch; ++beta)
                         if (beta < p.nb) slot[beta * tile_rows + hh * kRows + row] = ypart[hh][beta];
                 }
+            // Every thread's partial stores are fenced, then one counter increment (acquire and
+            // release at GPU scope) tells the last contributor that every partial is visible.
             __threadfence();
             if (!group_sync(ctl, gphase, lane, p)) break;
             if (gt == 0) {
-                const int old = atomicAdd(&p.tickets[gtile], 1);
+                int old;
+                asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(&p.tickets[gtile]) : "memory");
                 ctl->last = (old == lastc - first) ? 1 : 0;
             }
             if (!group_sync(ctl, gphase, lane, p)) break;
@@ -975,17 +1017,17 @@ struct Plan {
     uint32_t tmem_cols;
 };
 
-// Every A stage is filled by one expansion group only (so its phases stay in order).
-bool a_ring_owned(int n_a, int mh, int upp) {
-    int owner[kMaxAStages];
-    for (int s = 0; s < n_a; ++s) owner[s] = -1;
-    for (int i = 0; i < 4 * n_a; ++i)
-        for (int h = 0; h < mh; ++h)
-            for (int q = 0; q < upp; ++q) {
-                const int j = (i * mh + h) * upp + q, grp = a_group(i, h, q, mh, upp), s = j % n_a;
-                if (owner[s] >= 0 && owner[s] != grp) return false;
-                owner[s] = grp;
-            }
+// Every A stage serves one half only: its MMA issuers then consume its fills in order (an
+// issuer of the other half would wait on the phase after next, whose parity already reads as
+// complete).
+bool a_stages_per_half(int n_a, int mh, int upp) {
+    int half[kMaxAStages];
+    for (int s = 0; s < n_a; ++s) half[s] = -1;
+    for (int j = 0; j < 8 * n_a * mh * upp; ++j) {
+        const int s = j % n_a, h = (j / upp) % mh;
+        if (half[s] >= 0 && half[s] != h) return false;
+        half[s] = h;
+    }
     return true;
 }
 
@@ -1003,7 +1045,7 @@ bool plan_for(int P, bool f32x, int slice, Plan &L) {
     const int avail = 227 * 1024 - 1024 - static_cast<int>(sizeof(Ctl));
     for (int mh = 2; mh >= 1; --mh)
         for (int na = kMaxAStages; na >= 2; na -= 2) {
-            if (!a_ring_owned(na, mh, upp)) continue;
+            if (!a_stages_per_half(na, mh, upp)) continue;
             for (int n_acc = 2; n_acc >= 1; --n_acc) {
                 const int need = kSfCols + n_acc * mh * P * L.acc_stride + na * a_cols;
                 if (need > 512) continue;
@@ -1038,8 +1080,8 @@ inline int pairs_of(int K) { return (K + kPairCols - 1) / kPairCols; }
 inline size_t up1024(size_t v) { return (v + 1023) / 1024 * 1024; }
 
 struct WsLayout {
-    size_t off_tickets, off_inv, off_img, slice_bytes, total;
-    int tiles, slices;
+    size_t off_tickets, off_inv, off_bmax, off_img, slice_bytes, total;
+    int tiles, slices, maxblk;
 };
 
 WsLayout ws_layout(const GemvLayer *layers, int count, int P, const Plan &L, int batch) {
@@ -1052,8 +1094,11 @@ WsLayout ws_layout(const GemvLayer *layers, int count, int P, const Plan &L, int
     w.slices = (batch + L.slice - 1) / L.slice;
     w.slice_bytes = pair_rows * P * L.nm * 128;
     w.off_tickets = kPartialBytes;
+    for (int i = 0; i < count; ++i)
+        w.maxblk = std::max(w.maxblk, (pairs_of(layers[i].K) * kPairCols + kPrepCols - 1) / kPrepCols);
     w.off_inv = up1024(w.off_tickets + static_cast<size_t>(w.tiles) * sizeof(int));
-    w.off_img = up1024(w.off_inv + static_cast<size_t>(count) * P * batch * sizeof(float));
+    w.off_bmax = up1024(w.off_inv + static_cast<size_t>(count) * P * batch * sizeof(float));
+    w.off_img = up1024(w.off_bmax + static_cast<size_t>(count) * P * batch * w.maxblk * sizeof(float));
     w.total = w.off_img + w.slices * w.slice_bytes;
     return w;
 }
@@ -1092,12 +1137,15 @@ cudaError_t launch_gemv_group(const LaunchCtx &ctx, const GemvLayer *layers, int
     if (!encode) return cudaErrorNotSupported;
     void (*kern)(GArgs);
     void (*prep)(PrepArgs);
+    void (*bmax)(PrepArgs);
     if (P == 2) {
         kern = x_bf16 ? gemv_tc_kernel<false, 2> : gemv_tc_kernel<true, 2>;
         prep = x_bf16 ? gemv_prep_kernel<false, 2> : gemv_prep_kernel<true, 2>;
+        bmax = x_bf16 ? gemv_blockmax_kernel<false, 2> : gemv_blockmax_kernel<true, 2>;
     } else {
         kern = x_bf16 ? gemv_tc_kernel<false, 3> : gemv_tc_kernel<true, 3>;
         prep = x_bf16 ? gemv_prep_kernel<false, 3> : gemv_prep_kernel<true, 3>;
+        bmax = x_bf16 ? gemv_blockmax_kernel<false, 3> : gemv_blockmax_kernel<true, 3>;
     }
     static ContextFlags opted[4];
     // the opt-in is set once per kernel and context, to the largest size any call asks for
@@ -1127,6 +1175,8 @@ cudaError_t launch_gemv_group(const LaunchCtx &ctx, const GemvLayer *layers, int
         }
         pa.img = ws + W.off_img;
         pa.inv = reinterpret_cast<float *>(ws + W.off_inv);
+        pa.bmax = reinterpret_cast<float *>(ws + W.off_bmax);
+        pa.maxblk = W.maxblk;
         pa.tickets = reinterpret_cast<int *>(ws + W.off_tickets);
         pa.slice_bytes = static_cast<long long>(W.slice_bytes);
         pa.ntickets = W.tiles;
@@ -1145,6 +1195,7 @@ cudaError_t launch_gemv_group(const LaunchCtx &ctx, const GemvLayer *layers, int
         cfg.stream = ctx.stream;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        if (cudaError_t e = cudaLaunchKernelEx(&cfg, bmax, pa); e != cudaSuccess) return e;
         if (cudaError_t e = cudaLaunchKernelEx(&cfg, prep, pa); e != cudaSuccess) return e;
     }
 

@@ -99,16 +99,17 @@ PARTIAL_BYTES = 160 * 2 * 16 * 256 * 4     # partial sums: largest grid x 2 tile
 
 
 def test_gemv_workspace_layout(lib):
-    # partial sums, then the counters (4 bytes per 128-row tile) and the scales (4 bytes per
-    # path and batch row), each rounded up to 1 KiB, then the digit images: per 256 columns
-    # and path, 128 bytes per digit row (12 per batch row for fp32 x, rounded up to 8 rows)
-    assert lib.rabit_gemv_workspace_bytes(4096, 4096, 2, 1) == PARTIAL_BYTES + 1024 + 1024 + 16 * 2 * 16 * 128
-    assert lib.rabit_gemv_workspace_bytes(300, 1000, 3, 3) == PARTIAL_BYTES + 1024 + 1024 + 4 * 3 * 40 * 128
+    # partial sums, then the counters (4 bytes per row tile), the scales (4 bytes per path and
+    # batch row) and the block maxima (4 bytes per path, batch row and 1024 columns), each
+    # rounded up to 1 KiB, then the digit images: per 256 columns and path, 128 bytes per digit
+    # row (12 per batch row for fp32 x, rounded up to 8 rows)
+    assert lib.rabit_gemv_workspace_bytes(4096, 4096, 2, 1) == PARTIAL_BYTES + 3 * 1024 + 16 * 2 * 16 * 128
+    assert lib.rabit_gemv_workspace_bytes(300, 1000, 3, 3) == PARTIAL_BYTES + 3 * 1024 + 4 * 3 * 40 * 128
     for N, K, P, batch in [(1, 1, 2, 1), (14336, 4096, 2, 4), (4096, 11008, 2, 16), (4096, 4096, 3, 16)]:
         w = lib.rabit_gemv_workspace_bytes(N, K, P, batch)
         pairs = -(-K // 256)
         assert w >= PARTIAL_BYTES + 4 * -(-N // 128) + 4 * P * batch + pairs * P * 128 * 12 * batch
-        assert w <= PARTIAL_BYTES + 4 * -(-N // 128) + 2048 + 4 * P * batch + pairs * P * 128 * 24 * batch
+        assert w <= PARTIAL_BYTES + 4 * -(-N // 128) + 3072 + 4 * P * batch * (1 + pairs) + pairs * P * 128 * 24 * batch
     assert lib.rabit_gemv_workspace_bytes(8, 8, 2, 0) == 0
     assert lib.rabit_gemv_workspace_bytes(8, 8, 2, 17) == 0
 
@@ -192,7 +193,7 @@ def test_gemv_grouped_validation(lib):
         return ctypes.cast(a, ctypes.c_void_p)
     need = lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 2, 1, 1)
     # two one-tile, one-unit layers, bf16 x, batch 1: 8 digit rows of 128 bytes per path
-    assert need == PARTIAL_BYTES + 1024 + 1024 + 2 * 2 * 8 * 128
+    assert need == PARTIAL_BYTES + 3 * 1024 + 2 * 2 * 8 * 128
     assert lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 4, 1, 1) == 0
     assert lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 2, 7, 1) == 0
     assert lib.rabit_gemv_grouped_workspace_bytes(arr(), 2, 2, 1, 17) == 0
