@@ -970,7 +970,10 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
             if (ctl->last) {
                 __threadfence();
                 // The partials of contributors first..lastc, added in that (column) order.
-                // Loads go out eight at a time so their latencies overlap.
+                // Loads go out eight at a time so their latencies overlap.  Every contributor
+                // but the first starts its range inside this tile, so this tile is its first
+                // (slot 0); the first contributor's slot is 1 when its range starts earlier.
+                const int side_first = range_begin(U, G, first) < r.tile_begin ? 1 : 0;
                 for (int hh = 0; hh < mh; ++hh) {
                     const int tr = hh * kRows + row;
                     const int n = r.tile * tile_rows + tr;
@@ -983,7 +986,7 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
                                 const int i = i0 + dd;
                                 v[dd] = 0.0f;
                                 if (i <= lastc) {
-                                    const int si = (gtile == tile_of_unit(p, range_begin(U, G, i))) ? 0 : 1;
+                                    const int si = i == first ? side_first : 0;
                                     v[dd] = __ldcg(p.partial + ((static_cast<int64_t>(i) * 2 + si) * p.nb + beta) * tile_rows + tr);
                                 }
                             }
