@@ -38,6 +38,9 @@ int cuda_fail(cudaError_t e) {
     return RABIT_ERR_CUDA;
 }
 
+// Largest batch a single rabit_gemv call computes on the CUDA-core kernel by default.
+constexpr int kGemvCudaCoreMaxBatch = 4;
+
 bool env_flag(const char *name) {
     const char *v = std::getenv(name);
     return v && v[0] && std::strcmp(v, "0") != 0;
@@ -195,8 +198,16 @@ int rabit_gemv(const uint32_t *packed, const float *a, const float *b, int N, in
     uint32_t *fault = nullptr;
     int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
-    const char *which = std::getenv("RABIT_GEMV_KERNEL");
-    if (which && std::strcmp(which, "dp2a") == 0)
+    // Kernel choice.  A single layer at batch <= 4 goes to the CUDA-core kernel (gemv.cu): one
+    // launch with a small fixed cost, which decides at these sizes.  Larger batches go to the
+    // tensor-core path (gemv_tc.cu: prep kernels, then the sign stream on tcgen05), whose
+    // digit-sliced MMAs take all batch rows at once.  RABIT_GEMV_KERNEL=dp2a or =tc forces one.
+    bool tensor_cores = batch > kGemvCudaCoreMaxBatch;
+    if (const char *which = std::getenv("RABIT_GEMV_KERNEL")) {
+        if (std::strcmp(which, "dp2a") == 0) tensor_cores = false;
+        if (std::strcmp(which, "tc") == 0) tensor_cores = true;
+    }
+    if (!tensor_cores)
         return finish_launch(rabit::launch_gemv(ctx, packed, a, b, N, K, P, x, x_dtype == RABIT_BF16,
                                                 batch, ldx, y, ldy, fault, wait_timeout_ns()));
     const int debug = env_flag("RABIT_TEST_GEMV_WITHHOLD_COPY") ? 2 : 0;

@@ -104,11 +104,17 @@ RABIT_API int rabit_derive_pack(const void *W, int w_dtype, int N, int K, int ld
  * Appendix E.1 "Compute Pipeline": paths computed in parallel, signs applied without
  * multiplication, output scale applied last):
  *     y[beta][n] = sum_k a[k][n] * sum_j S_k[n][j] * b[k][j] * x[beta][j]
- * The signs enter the tensor cores as 4-bit +-1 values and the activation term
- * z = b_k * x (an fp32 product) as balanced base-4 digits of zq = rint(z * 2^e): one
- * power-of-two scale per (path, batch row) puts |zq| below 2^15 (bf16 x) or 2^23 (fp32 x).
- * The sign sums of zq are exact; results are deterministic.  Two kernels run on `stream`:
- * one prepares the digits and scales in the workspace, the other streams the signs.
+ * Two implementations, chosen by batch (RABIT_GEMV_KERNEL=dp2a or =tc in the environment
+ * forces one):
+ *   batch <= 4: one CUDA-core kernel.  z = b_k * x is quantised per 32-column group to 13
+ *     bits (two 13-bit slices for fp32 x) with a power-of-two scale; the signs select which
+ *     z enter integer dot products (dp2a), exact in 32-bit.
+ *   batch > 4 (and every rabit_gemv_grouped call): the tensor-core path.  The signs enter
+ *     tcgen05.mma as 4-bit +-1 values and z as balanced base-4 digits of zq = rint(z * 2^e)
+ *     with one power-of-two scale per (path, batch row), |zq| below 2^15 (bf16 x) or 2^23
+ *     (fp32 x); the sign sums of zq are exact.  Prep kernels write the digits and scales
+ *     to the workspace, then the main kernel streams the signs.
+ * Results are deterministic.
  *   packed  RABIT_LAYOUT_V2 buffer of N x K, P paths (input)
  *   a [P][N], b [P][K] fp32
  *   x       [batch][ldx], bf16 (x_dtype RABIT_BF16) or fp32 (RABIT_F32), ldx >= K

@@ -93,6 +93,7 @@ def test_gemv_copy_wait_expiry_is_reported_and_the_context_survives(monkeypatch,
     W, a, b, x, at, bt, packed, xt = _case(N, K, batch, seed=4300 + N)
     ws = rabit.alloc_gemv_workspace(N, K, 2, batch)
     y = torch.zeros((batch, N), device="cuda")
+    monkeypatch.setenv("RABIT_GEMV_KERNEL", "tc")     # the tensor-core path has the copy waits
     monkeypatch.setenv("RABIT_TEST_GEMV_WITHHOLD_COPY", "1")
     monkeypatch.setenv("RABIT_WAIT_TIMEOUT_MS", "50")
     rabit.rabit_gemv(packed, at, bt, N, K, xt, y, workspace=ws)

@@ -122,12 +122,19 @@ def test_derive_pack_hand_cases(golden_dir):
 
 
 # ------------------------------------------------------------------ gemv
+@pytest.fixture(params=["tc", "dp2a"])
+def gemv_kernel(request, monkeypatch):
+    """Both decode implementations: rabit_gemv picks one by batch; the environment forces it."""
+    monkeypatch.setenv("RABIT_GEMV_KERNEL", request.param)
+    return request.param
+
+
 GEMV_SHAPES = [(1, 1), (32, 128), (33, 129), (96, 1000), (300, 520), (1024, 4096)]
 
 
 @pytest.mark.parametrize("N,K", GEMV_SHAPES)
 @pytest.mark.parametrize("batch", [1, 2, 3, 8, 16])
-def test_gemv_bf16_matches_oracle(N, K, batch):
+def test_gemv_bf16_matches_oracle(N, K, batch, gemv_kernel):
     W, a, b = make_layer(200 + N, N, K)
     S = oracle.derive_signs(W, a, b)
     packed = dev(oracle.pack(S))
@@ -141,7 +148,7 @@ def test_gemv_bf16_matches_oracle(N, K, batch):
 
 @pytest.mark.parametrize("N,K", [(33, 129), (300, 520), (1024, 4096)])
 @pytest.mark.parametrize("batch", [1, 5])
-def test_gemv_fp32_matches_oracle(N, K, batch):
+def test_gemv_fp32_matches_oracle(N, K, batch, gemv_kernel):
     W, a, b = make_layer(300 + N, N, K)
     S = oracle.derive_signs(W, a, b)
     packed = dev(oracle.pack(S))
@@ -156,7 +163,7 @@ def test_gemv_fp32_matches_oracle(N, K, batch):
 @pytest.mark.parametrize("P", [2, 3])
 @pytest.mark.parametrize("N,K,batch", [(300, 520, 2), (300, 520, 7), (1024, 4096, 4), (4096, 4096, 6),
                                        (1000, 1000, 16)])
-def test_gemv_each_batch_row_matches_oracle(N, K, batch, P):
+def test_gemv_each_batch_row_matches_oracle(N, K, batch, P, gemv_kernel):
     """Batch rows of magnitudes 2^-6 .. 2^+6 apart: every row is checked on its own, so a row
     scaled with another row's z scale, or left unwritten, fails."""
     W, a, b = make_layer(400 + N + batch, N, K)
@@ -176,7 +183,7 @@ def test_gemv_each_batch_row_matches_oracle(N, K, batch, P):
         assert normwise(yh[beta], ref[beta]) <= TOL_BF16, beta
 
 
-def test_gemv_pitched_io():
+def test_gemv_pitched_io(gemv_kernel):
     N, K, batch = 70, 300, 4
     W, a, b = make_layer(9, N, K)
     S = oracle.derive_signs(W, a, b)

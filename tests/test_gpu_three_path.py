@@ -51,6 +51,13 @@ def layer3(seed, N, K, w_bf16=False):
     return S, a, b, at, bt, packed
 
 
+@pytest.fixture(params=["tc", "dp2a"])
+def gemv_kernel(request, monkeypatch):
+    """Both decode implementations (rabit_gemv picks one by batch; the environment forces it)."""
+    monkeypatch.setenv("RABIT_GEMV_KERNEL", request.param)
+    return request.param
+
+
 @pytest.mark.parametrize("N,K,w_bf16", [(33, 129, False), (300, 520, True), (1024, 4096, False)])
 def test_derive_pack_three_paths_bit_exact(N, K, w_bf16):
     S, a, b, at, bt, packed = layer3(80 + N, N, K, w_bf16)
@@ -58,7 +65,7 @@ def test_derive_pack_three_paths_bit_exact(N, K, w_bf16):
 
 
 @pytest.mark.parametrize("N,K,batch", [(33, 129, 1), (300, 520, 3), (1024, 4096, 1), (4096, 4096, 4)])
-def test_gemv_three_paths_bf16(N, K, batch):
+def test_gemv_three_paths_bf16(N, K, batch, gemv_kernel):
     S, a, b, at, bt, packed = layer3(81 + N, N, K)
     x = inputs.activations(81 + N, batch, K)
     y = torch.empty((batch, N), device="cuda")
@@ -69,7 +76,7 @@ def test_gemv_three_paths_bf16(N, K, batch):
 
 
 @pytest.mark.parametrize("N,K,batch", [(33, 129, 1), (300, 520, 5)])
-def test_gemv_three_paths_fp32(N, K, batch):
+def test_gemv_three_paths_fp32(N, K, batch, gemv_kernel):
     S, a, b, at, bt, packed = layer3(82 + N, N, K)
     x = inputs.activations(82 + N, batch, K, dtype="f32")
     y = torch.empty((batch, N), device="cuda")
