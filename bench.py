@@ -60,7 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=400)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the GEMM / derive / CPU-baseline measurements")
-    ap.add_argument("--profile-kernel", choices=["derive", "gemv", "gemm", "svid"], default=None,
+    ap.add_argument("--profile-kernel", choices=["derive", "gemv", "gemv_set", "gemm", "svid"], default=None,
                     help="run a few launches of one kernel (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=3, metavar=("N", "K", "M"), default=(11008, 4096, 1),
                     help="with --profile-kernel: out features, in features, batch/tokens")
@@ -178,28 +178,6 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-# Compute bound of the decode kernel.  It feeds the sign bits to tcgen05.mma kind::i8 as one
-# byte each (the A operand, 128 rows x 32 bytes per instruction), and at M = 128 with N <= 64
-# one such instruction takes 44.8 SM clocks whatever N is (measured on this part; N = 256
-# takes 128 clocks, the full i8 rate).  So the tensor core takes in at most 4096 / 44.8 =
-# 91.4 sign bits per clock per SM, at every batch size up to 16.
-TC_SIGN_BITS_PER_SM_CLK = 91.4
-
-
-def tc_peak_gbs(device) -> tuple[float, str]:
-    """Decode compute bound in GB/s of packed sign bits: SMs x max SM clock x 91.4 bits / 8."""
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    mhz = 1965.0
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            mhz = float(json.load(f).get("sm_max_mhz", mhz))
-    except Exception:
-        pass
-    return (sms * mhz * 1e6 * TC_SIGN_BITS_PER_SM_CLK / 8 / 1e9,
-            f"{sms} SMs x {mhz:.0f} MHz x {TC_SIGN_BITS_PER_SM_CLK} sign bits/clk "
-            "(A-operand intake of tcgen05.mma kind::i8 at M=128, N<=64)")
-
-
 def sign_bytes(layers) -> int:
     """Packed sign bytes of one decode pass (the work of the dp2a pipe)."""
     return sum(2 * L["N"] * (((L["K"] + 127) // 128) * 128) // 8 for L in layers)
@@ -222,6 +200,46 @@ def make_layer(rabit, spec, idx, name, N, K, device, batch, P=2):
     return dict(name=name, N=N, K=K, P=P, a=at, b=bt, packed=packed, x_host=x,
                 x=bf16_tensor(x, device), y=torch.empty((batch, N), device=device),
                 ws=rabit.alloc_gemv_workspace(N, K, P, min(batch, 16), device=device) if batch <= 16 else None)
+
+
+def layer_tuples(layers, B=None):
+    """(packed, a, b, N, K, x, y) of each layer for rabit_gemv_grouped (first B batch rows)."""
+    return [(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"][:B] if B else L["x"],
+             L["y"][:B] if B else L["y"]) for L in layers]
+
+
+# Decoder-order grouping of each decode set: the projections that read the same activation
+# share one call (q, k, v; gate, up); o and down each follow their own input.
+DECODER_GROUPS = {"llama2_7b_decode_b1": [[0, 1, 2], [3], [4, 5], [6]],
+                  "llama3_8b_decode": [[0, 1, 2], [3, 4], [5]]}
+
+
+def decode_schedules(rabit, sets, spec_name, device, B=None, steps=400, warmup=20):
+    """Microseconds per set for three schedules of the same matrices: one rabit_gemv per matrix
+    (the library picks the kernel by batch), one rabit_gemv_grouped per decoder group, and one
+    rabit_gemv_grouped over the whole set (the matrices as independent GEMVs)."""
+    base = sets[0]
+    ws = rabit.alloc_gemv_grouped_workspace(layer_tuples(base, B), P=base[0]["P"], device=device)
+    groups = DECODER_GROUPS[spec_name]
+
+    def per_matrix(ls):
+        return lambda: [rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"],
+                                         L["x"][:B] if B else L["x"], L["y"][:B] if B else L["y"],
+                                         P=L["P"], workspace=L["ws"]) for L in ls]
+
+    def grouped(ls):
+        return lambda: [rabit.rabit_gemv_grouped(layer_tuples([ls[i] for i in g], B), P=ls[0]["P"], workspace=ws)
+                        for g in groups]
+
+    def one_call(ls):
+        return lambda: rabit.rabit_gemv_grouped(layer_tuples(ls, B), P=ls[0]["P"], workspace=ws)
+
+    out = {}
+    for name, mk in (("per_matrix", per_matrix), ("decoder_groups", grouped), ("one_call", one_call)):
+        graphs = [capture_graph(mk(ls)) for ls in sets]
+        out[name] = round(timed_replays(graphs, steps, warmup, None, device) / steps * 1e3, 2)
+        del graphs
+    return out
 
 
 def decode_bytes(layers, batch=1):
@@ -345,10 +363,11 @@ def measure_fp8_tflops(device, n=8192, reps=10):
         return None
 
 
-def bench_decode_sweep(rabit, device, tc_peak, hbm_peak):
+def bench_decode_sweep(rabit, device, hbm_peak):
     """Llama-3-8B-shaped decode set (q 4096x4096, k/v 1024x4096, gate/up 14336x4096, down
-    4096x14336, 0.1% x20 weight outliers) at batch 1, 4, 8 and 16: microseconds per set and per
-    layer, three rotated copies of the packed weights (more than L2)."""
+    4096x14336, 0.1% x20 weight outliers) at batch 1, 4, 8 and 16: microseconds per set for the
+    per-matrix, decoder-order and one-call schedules, three rotated copies of the packed
+    weights (more than L2)."""
     spec = inputs.WORKLOADS["llama3_8b_decode"]
     out = {"workload": "llama3_8b_decode", "copies": 3, "by_batch": {}}
     Bmax = max(spec["batches"])
@@ -356,27 +375,12 @@ def bench_decode_sweep(rabit, device, tc_peak, hbm_peak):
             for idx, (name, N, K) in enumerate(spec["set"])]
     sets = [base] + [[dict(L, packed=L["packed"].clone()) for L in base] for _ in range(2)]
     torch.cuda.synchronize()
-    sign = sign_bytes(base)
     for B in spec["batches"]:
-        def step_fn(layers, B=B):
-            def f():
-                for L in layers:
-                    rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"][:B], L["y"][:B],
-                                     workspace=L["ws"])
-            return f
-
-        graphs = [capture_graph(step_fn(ls)) for ls in sets]
-        steps = 600
-        ms = timed_replays(graphs, steps, 30, None, device)
-        us = ms / steps * 1e3
+        sched = decode_schedules(rabit, sets, "llama3_8b_decode", device, B=B, steps=300, warmup=20)
         byts = decode_bytes(base, batch=B)
-        out["by_batch"][str(B)] = {
-            "us_per_set": round(us, 2), "us_per_layer": round(us / len(base), 2),
-            "GB_per_s": round(byts / (us * 1e-6) / 1e9, 1),
-            "hbm_frac": round(byts / (us * 1e-6) / 1e9 / hbm_peak, 4),
-            # the tensor core takes each sign bit in once for all B batch rows (N <= 64)
-            "tensor_frac": round(sign / (us * 1e-6) / 1e9 / tc_peak, 4)}
-        del graphs
+        out["by_batch"][str(B)] = {k: {"us_per_set": v, "GB_per_s": round(byts / (v * 1e-6) / 1e9, 1),
+                                       "hbm_frac": round(byts / (v * 1e-6) / 1e9 / hbm_peak, 4)}
+                                   for k, v in sched.items()}
     del sets, base
     torch.cuda.empty_cache()
     return out
@@ -398,7 +402,7 @@ def warm_launch_us(rabit, layers, device):
     return out
 
 
-def bench_gemv_three_path(rabit, device, tc_peak, hbm_peak):
+def bench_gemv_three_path(rabit, device, hbm_peak):
     """The 3-bit variant (three paths) on the same Llama-2-7B decode set, batch 1, ten rotated
     copies (the pages' Table 7 reports 3-bit kernel latencies beside the 2-bit ones)."""
     spec = inputs.WORKLOADS[WORKLOAD]
@@ -406,29 +410,16 @@ def bench_gemv_three_path(rabit, device, tc_peak, hbm_peak):
             for idx, (name, N, K) in enumerate(spec["set"])]
     sets = [base] + [[dict(L, packed=L["packed"].clone()) for L in base] for _ in range(COPIES - 1)]
     torch.cuda.synchronize()
-
-    def step_fn(layers):
-        def f():
-            for L in layers:
-                rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"], P=3,
-                                 workspace=L["ws"])
-        return f
-
-    graphs = [capture_graph(step_fn(ls)) for ls in sets]
-    steps = 2000
-    ms = timed_replays(graphs, steps, 50, None, device)
-    sign = sum(3 * L["N"] * (((L["K"] + 127) // 128) * 128) // 8 for L in base)
+    sched = decode_schedules(rabit, sets, WORKLOAD, device, steps=1000, warmup=50)
     algo = sum(3 * L["N"] * (((L["K"] + 127) // 128) * 128) // 8 + 4 * 3 * (L["N"] + L["K"])
                + L["K"] * 2 + L["N"] * 4 for L in base)
-    return {"workload": "llama2_7b_decode_b1_3path", "value": round(algo * steps / (ms * 1e-3) / 1e9, 1),
-            "unit": "GB/s", "us_per_set": round(ms / steps * 1e3, 2),
+    best = sched["one_call"]
+    gbs = algo / (best * 1e-6) / 1e9
+    return {"workload": "llama2_7b_decode_b1_3path", "value": round(gbs, 1), "unit": "GB/s",
+            "us_per_set": best, "schedules_us_per_set": sched,
             "us_per_launch_warm_l2_by_shape": warm_launch_us(rabit, base, device),
-            "roofline": {"bound": "hbm", "achieved": round(algo * steps / (ms * 1e-3) / 1e9, 1),
-                         "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(algo * steps / (ms * 1e-3) / 1e9 / hbm_peak, 4)},
-            "roofline_compute": {"bound": "tensor", "achieved": round(sign * steps / (ms * 1e-3) / 1e9, 1),
-                                 "peak": round(tc_peak, 1), "unit": "GB/s",
-                                 "frac": round(sign * steps / (ms * 1e-3) / 1e9 / tc_peak, 4)},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4)},
             "note": "3 sign words + 1 padding word per group in HBM; algorithmic bytes count the 3 signs"}
 
 
@@ -707,10 +698,13 @@ def run_ours(args, rank, world, local, dist):
     torch.cuda.synchronize()
     step_bytes = decode_bytes(base)
 
+    # One step: the seven matrices of the set as one rabit_gemv_grouped call (three kernels:
+    # block maxima, digit images, the sign stream on the tensor cores).
+    ws = rabit.alloc_gemv_grouped_workspace(layer_tuples(base), device=device)
+
     def step_fn(layers):
         def f():
-            for L in layers:
-                rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"])
+            rabit.rabit_gemv_grouped(layer_tuples(layers), workspace=ws)
         return f
 
     graphs = [capture_graph(step_fn(ls)) for ls in sets]
@@ -718,11 +712,9 @@ def run_ours(args, rank, world, local, dist):
     elapsed_ms = timed_replays(graphs, args.steps, args.warmup, dist, device, clocks)
     max_ms, total_units = aggregate(elapsed_ms, float(step_bytes) * args.steps, dist, device)
     value = total_units / (max_ms * 1e-3) / 1e9
-    launches = len(base) * args.steps
-    per_launch_us = elapsed_ms * 1e3 / launches
+    launches = 3 * args.steps
+    per_call_us = elapsed_ms * 1e3 / args.steps
     achieved = step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
-    tc_peak, tc_kind = tc_peak_gbs(device)
-    tc_achieved = sign_bytes(base) * args.steps / (elapsed_ms * 1e-3) / 1e9
     # every bounded device wait of the timed region must have completed
     fault = rabit.rabit_read_fault(clear=True)
 
@@ -736,9 +728,10 @@ def run_ours(args, rank, world, local, dist):
 
     def e2e_step(s):
         layers = sets[s % COPIES]
-        for L, xp, yp in zip(layers, x_pinned, y_pinned):
+        for L, xp in zip(layers, x_pinned):
             L["x"].copy_(xp, non_blocking=True)
-            rabit.rabit_gemv(L["packed"], L["a"], L["b"], L["N"], L["K"], L["x"], L["y"], workspace=L["ws"])
+        rabit.rabit_gemv_grouped(layer_tuples(layers), workspace=ws)
+        for L, yp in zip(layers, y_pinned):
             yp.copy_(L["y"], non_blocking=True)
         stream.synchronize()
 
@@ -765,29 +758,34 @@ def run_ours(args, rank, world, local, dist):
                    "weights": "2-path packed signs derived on the GPU from seeded fp32 W ~ N(0, 0.02^2)",
                    "l2": f"inputs larger than L2: {COPIES} resident copies of the layer set "
                          f"({COPIES * step_bytes / 1e6:.0f} MB) rotated per step",
+                   "schedule": "the 7 matrices as one rabit_gemv_grouped call per step (independent GEMVs, "
+                               "each with its own seeded x); per-matrix and decoder-order schedules in "
+                               "decode_schedules",
                    "launch": "CUDA graph per copy, programmatic dependent launch between kernels",
                    "parallelism": f"replica x{world}"},
         # The metric's "% of peak": algorithmic bytes of the decode pass over the measured HBM
-        # copy bandwidth.  The tensor core's intake of sign bits (TC_SIGN_BITS_PER_SM_CLK) is the
-        # compute bound beside it.
+        # copy bandwidth, per call of the hot path (its three kernels, chained).
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                     "kernel": "gemv_tc_kernel", "avg_launch_us": round(per_launch_us, 3),
+                     "kernel": "gemv_tc_kernel (+ gemv_blockmax_kernel, gemv_prep_kernel)",
+                     "avg_call_us": round(per_call_us, 3),
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                     "achieved_kind": "algorithmic bytes (signs, scales, x, y) per launch / average launch time"},
-        "roofline_compute": {"bound": "tensor", "achieved": round(tc_achieved, 2), "peak": round(tc_peak, 1),
-                             "unit": "GB/s", "frac": round(tc_achieved / tc_peak, 4), "peak_kind": tc_kind,
-                             "achieved_kind": "packed sign bytes per second"},
+                     "achieved_kind": "algorithmic bytes (signs, scales, x, y) per call / average call time"},
         "gpu_launches": launches,
         "fault_word": fault,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "api": "bit_gemv_rabit_b200.rabit.rabit_gemv per matrix, pinned host copies, stream sync per step"},
+                "api": "bit_gemv_rabit_b200.rabit.rabit_gemv_grouped over the set, pinned host copies, "
+                       "stream sync per step"},
     }
     if clocks is not None:
         line["clocks"] = clocks.summary()
     if rank == 0 and world == 1 and not args.no_secondary:
         line["us_per_launch_warm_l2_by_shape"] = warm_launch_us(rabit, base, device)
+        sched = decode_schedules(rabit, sets, WORKLOAD, device)
+        line["decode_schedules"] = {k: {"us_per_set": v, "GB_per_s": round(step_bytes / (v * 1e-6) / 1e9, 1),
+                                        "hbm_frac": round(step_bytes / (v * 1e-6) / 1e9 / hbm_peak, 4)}
+                                    for k, v in sched.items()}
     traffic = _load_traffic()
     if traffic is not None:
         line["roofline"]["traffic"] = traffic
@@ -798,10 +796,10 @@ def run_ours(args, rank, world, local, dist):
         secondary(line, "gemm", lambda: bench_gemm(rabit, device, hbm_peak, tf_peak, tf_sustained))
         secondary(line, "qat_step", lambda: bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained),
                   merge=True)
-        secondary(line, "gemv_3path", lambda: bench_gemv_three_path(rabit, device, tc_peak, hbm_peak))
+        secondary(line, "gemv_3path", lambda: bench_gemv_three_path(rabit, device, hbm_peak))
         secondary(line, "scale_grads", lambda: bench_scale_grads(rabit, device, hbm_peak))
         secondary(line, "svid_init", lambda: bench_svid_init(rabit, device, hbm_peak))
-        secondary(line, "decode_batch_sweep", lambda: bench_decode_sweep(rabit, device, tc_peak, hbm_peak))
+        secondary(line, "decode_batch_sweep", lambda: bench_decode_sweep(rabit, device, hbm_peak))
     if rank == 0:
         # parity of the timed configuration: every output of the last timed step against the
         # float64 oracle (normwise, per matrix; the bar is 2e-3 for bf16 activations)
@@ -846,10 +844,21 @@ def secondary(line, key, fn, merge=False):
 
 
 def profile_kernel(args):
-    """A few launches of one kernel on a seeded layer of the given shape (ncu target)."""
+    """A few launches of one kernel on a seeded layer of the given shape (ncu target); with
+    gemv_set, --launches grouped calls over the benchmark's decode layer set."""
     from bit_gemv_rabit_b200 import rabit
     rabit.load()
     device = torch.device("cuda", 0)
+    if args.profile_kernel == "gemv_set":
+        spec = inputs.WORKLOADS[WORKLOAD]
+        layers = [make_layer(rabit, spec, idx, name, N, K, device, 1) for idx, (name, N, K) in enumerate(spec["set"])]
+        ws = rabit.alloc_gemv_grouped_workspace(layer_tuples(layers), device=device)
+        for _ in range(args.launches):
+            rabit.rabit_gemv_grouped(layer_tuples(layers), workspace=ws)
+        torch.cuda.synchronize()
+        fault = rabit.rabit_read_fault()
+        print(f"gemv_set {WORKLOAD} launches={args.launches} fault={fault}")
+        return 0 if fault == 0 else 1
     N, K, M = args.shape
     spec = dict(cfg=9, sigma=0.02, w_outliers=0.0, x_outliers=0.0)
     L = make_layer(rabit, spec, 0, "layer", N, K, device, M)
