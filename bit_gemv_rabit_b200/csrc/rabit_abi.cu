@@ -275,6 +275,25 @@ int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, in
                                             workspace, fault, timeout_ns, debug));
 }
 
+int rabit_transpose_pack(const uint32_t *packed, int N, int K, int P, uint32_t *packed_t, void *stream) {
+    if (!packed || !packed_t) return RABIT_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || P < 1) return RABIT_ERR_SHAPE;
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16) || !aligned(packed_t, 16)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    int st = device_ctx(stream, ctx, nullptr);
+    if (st != RABIT_OK) return st;
+    return finish_launch(rabit::launch_transpose_pack(ctx, packed, N, K, P, packed_t));
+}
+
+// The input gradient is the forward GEMM of the transposed layer: signs S_k^T (K x N), the
+// per-output scale b_k (length K) and the per-input scale a_k (length N), activations dY.
+int rabit_grad_x(const uint32_t *packed_t, const float *a, const float *b, int N, int K, int P,
+                 const uint16_t *dy_bf16, int M, int ldd, float *grad_x, int ldg, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    return rabit_gemm(packed_t, b, a, K, N, P, dy_bf16, M, ldd, grad_x, ldg, workspace, workspace_bytes, stream);
+}
+
 // For callers that may not allocate device memory: the scratch comes from the library's
 // fixed buffer instead of a caller workspace (see include/rabit.h).
 int rabit_gemm_noalloc(const uint32_t *packed, const float *a, const float *b, int N, int K, int P,

@@ -67,6 +67,10 @@ cudaError_t launch_gemv_tc(const LaunchCtx &ctx, const uint32_t *packed, const f
                            int N, int K, int P, const void *x, bool x_bf16, int batch, int ldx, float *y,
                            int ldy, void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug);
 
+// Packed sign planes of W^T (K x N) from those of W (transpose_pack.cu).
+cudaError_t launch_transpose_pack(const LaunchCtx &ctx, const uint32_t *packed, int N, int K, int P,
+                                  uint32_t *packed_t);
+
 // The driver's cuTensorMapEncodeTiled (as a PFN_cuTensorMapEncodeTiled_v12000), or null.
 void *tensor_map_encode_entry();
 

@@ -32,6 +32,8 @@ SIGNATURES = [
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_gemm_noalloc", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p]),
+    ("rabit_transpose_pack", _i, [_p, _i, _i, _i, _p, _p]),
+    ("rabit_grad_x", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_scale_grads_workspace_bytes", _sz, [_i, _i, _i]),
     ("rabit_scale_grads", _i, [_p, _i, _p, _p, _p, _i, _i, _i, _p, _p, _p, _sz, _p]),
     ("rabit_svid_init_workspace_bytes", _sz, [_i, _i, _i]),
@@ -189,6 +191,27 @@ def rabit_gemm(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K
                              _dptr(y), y.stride(0), _dptr(workspace), ws_bytes, _stream(stream)),
            "rabit_gemm")
     return y
+
+
+def rabit_transpose_pack(packed: torch.Tensor, N: int, K: int, packed_t: torch.Tensor, P: int = 2,
+                         stream=None) -> torch.Tensor:
+    """packed: signs of N x K; packed_t (alloc_packed(K, N, P)) receives those of the transpose."""
+    _check(load().rabit_transpose_pack(_dptr(packed), N, K, P, _dptr(packed_t), _stream(stream)),
+           "rabit_transpose_pack")
+    return packed_t
+
+
+def rabit_grad_x(packed_t: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,
+                 dy: torch.Tensor, grad_x: torch.Tensor, workspace: torch.Tensor, P: int = 2,
+                 stream=None) -> torch.Tensor:
+    """dy [M][N] bf16; grad_x [M][K] fp32 out; packed_t from rabit_transpose_pack; workspace
+    from alloc_gemm_workspace(K, N, P, M)."""
+    M = dy.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().rabit_grad_x(_dptr(packed_t), _dptr(a), _dptr(b), N, K, P, _dptr(dy), M, dy.stride(0),
+                               _dptr(grad_x), grad_x.stride(0), _dptr(workspace), ws_bytes, _stream(stream)),
+           "rabit_grad_x")
+    return grad_x
 
 
 def rabit_gemm_noalloc(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,

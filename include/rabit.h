@@ -191,6 +191,36 @@ RABIT_API int rabit_gemm(const uint32_t *packed, const float *a, const float *b,
                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * rabit_transpose_pack -- the packed sign planes of W^T from those of W, for the input
+ * gradient (sec. 4.1: W_hat = sum_k a_k (.) S_k (.) b_k, so W_hat^T = sum_k b_k (.) S_k^T (.) a_k
+ * is a stacked layer of the same form, K x N, with a and b exchanged):
+ *     packed_t holds S_k^T[j][n] = S_k[n][j] for every path k, j < K, n < N.
+ *   packed    RABIT_LAYOUT_V2 buffer of N x K, P paths (input)
+ *   packed_t  RABIT_LAYOUT_V2 buffer of K x N, P paths: rabit_packed_words(K, N, P) uint32,
+ *             16-byte aligned (output, every word written, padding columns n >= N zero)
+ * Bit-exact.  Errors: INVALID_ARG, SHAPE, UNSUPPORTED (P not 2 or 3), ALIGNMENT, ARCH, CUDA.
+ */
+RABIT_API int rabit_transpose_pack(const uint32_t *packed, int N, int K, int P, uint32_t *packed_t,
+                                   void *stream);
+
+/*
+ * rabit_grad_x -- input gradient of the layer for M tokens (the backward of sec. 4.1's
+ * stacked layer with the signs held fixed):
+ *     grad_x[m][j] = sum_n dY[m][n] W_hat[n][j] = sum_k b_k[j] sum_n S_k[n][j] a_k[n] dY[m][n]
+ * computed as rabit_gemm of the transposed layer: signs from rabit_transpose_pack, per-output
+ * scale b_k, per-input scale a_k, activations dY (on tcgen05, fp32 accumulation).
+ *   packed_t  RABIT_LAYOUT_V2 of K x N from rabit_transpose_pack (input)
+ *   a [P][N], b [P][K] fp32 (the layer's scales, as for rabit_gemm)
+ *   dy_bf16   [M][ldd] bf16, ldd >= N and a multiple of 8, 16-byte aligned
+ *   grad_x    [M][ldg] fp32 (output), ldg >= K
+ *   workspace at least rabit_gemm_workspace_bytes(K, N, P, M) bytes, 256-byte aligned
+ * Accuracy (normwise): <= 2e-3, the bar of rabit_gemm.  Errors: those of rabit_gemm.
+ */
+RABIT_API int rabit_grad_x(const uint32_t *packed_t, const float *a, const float *b, int N, int K, int P,
+                           const uint16_t *dy_bf16, int M, int ldd, float *grad_x, int ldg,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * rabit_gemm_noalloc -- the same computation as rabit_gemm, for callers that are not allowed
  * to allocate device memory and so cannot hand rabit_gemm a workspace.  Examples: a plugin
  * loaded into an inference engine that owns every device allocation and gives the plugin

@@ -59,6 +59,8 @@ def _load():
         lib.oracle_layer.restype = None
         lib.oracle_scale_grads.argtypes = [p, i64, i64, p, ctypes.c_int, p, p, p, p]
         lib.oracle_scale_grads.restype = None
+        lib.oracle_grad_x.argtypes = [p, i64, i64, ctypes.c_int, p, p, p, i64, i64, p]
+        lib.oracle_grad_x.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -172,3 +174,27 @@ def scale_grads(G: np.ndarray, S: np.ndarray, a: np.ndarray, b: np.ndarray):
     gb = np.empty((P, K), dtype=np.float64)
     _load().oracle_scale_grads(_ptr(Gd), N, K, _ptr(S), P, _ptr(ad), _ptr(bd), _ptr(ga), _ptr(gb))
     return ga, gb
+
+
+def grad_x(S: np.ndarray, a: np.ndarray, b: np.ndarray, dY: np.ndarray,
+           cols: np.ndarray | None = None) -> np.ndarray:
+    """Input gradient of sec. 4.1's stacked layer with the signs held fixed:
+    gx[m][c] = sum_n dY[m][n] W_hat[n][j_c], W_hat = sum_k a_k S_k b_k.
+
+    S: int8 [P][N][C], the signs of the C columns j_c (cols, or all K columns when cols is
+    None); a: [P][N]; b: [P][K]; dY: [M][N] (float32, float64 or bf16 bits).
+    Returns float64 [M][C]."""
+    S = np.ascontiguousarray(S, dtype=np.int8)
+    P, N, C = S.shape
+    ad = np.ascontiguousarray(widen(a)).reshape(-1, N)
+    bd = np.ascontiguousarray(widen(b)).reshape(P, -1)
+    bc = np.ascontiguousarray(bd if cols is None else bd[:, np.asarray(cols)])
+    assert bc.shape == (P, C)
+    dYd = np.ascontiguousarray(widen(dY))
+    if dYd.ndim == 1:
+        dYd = dYd[None, :]
+    M = dYd.shape[0]
+    assert dYd.shape[1] == N
+    gx = np.empty((M, C), dtype=np.float64)
+    _load().oracle_grad_x(_ptr(S), N, C, P, _ptr(ad), _ptr(bc), _ptr(dYd), M, N, _ptr(gx))
+    return gx

@@ -183,6 +183,34 @@ ORACLE_API void oracle_scale_grads(const double *G, int64_t N, int64_t K, const 
     }
 }
 
+/*
+ * Input gradient of the stacked layer (sec. 4.1) with the signs held fixed: for
+ * y = W_hat x with W_hat[n][j] = sum_k a_k[n] S_k[n][j] b_k[j],
+ *   gx[m][c] = dL/dx[m][j_c] = sum_n dY[m][n] W_hat[n][j_c]
+ *            = sum_k b_k[j_c] sum_n dY[m][n] a_k[n] S_k[n][c]
+ *   S  : int8 [P][N][C], the signs of the C columns j_c (all rows n)
+ *   a  : [P][N];  bc : [P][C] (b_k at the C columns);  dY : float64 [M][ldd]
+ *   gx : float64 [M][C]
+ */
+ORACLE_API void oracle_grad_x(const int8_t *S, int64_t N, int64_t C, int P, const double *a,
+                              const double *bc, const double *dY, int64_t M, int64_t ldd, double *gx)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t c = 0; c < C; ++c) {
+            double acc = 0.0;
+            for (int k = 0; k < P; ++k) {
+                const int8_t *Sk = S + (int64_t)k * N * C;
+                double t = 0.0;
+                for (int64_t n = 0; n < N; ++n)
+                    t += dY[m * ldd + n] * a[(int64_t)k * N + n] * (double)Sk[n * C + c];
+                acc += bc[(int64_t)k * C + c] * t;
+            }
+            gx[m * C + c] = acc;
+        }
+    }
+}
+
 /* Number of OpenMP threads the parallel loops above use (1 without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

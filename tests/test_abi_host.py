@@ -210,3 +210,20 @@ def test_gemv_grouped_validation(lib):
     assert f(arr(), 2, 4, 1, 1, P(FAKE), need, None) == UNSUP
     assert f(arr(), 2, 2, 1, 1, P(FAKE), need - 1, None) == WS
     assert f(arr(), 2, 2, 1, 1, P(FAKE + 8), need, None) == ALIGN
+
+
+def test_transpose_pack_and_grad_x_validation(lib):
+    f = lib.rabit_transpose_pack
+    assert f(None, 4, 4, 2, P(FAKE), None) == INVALID
+    assert f(P(FAKE), 0, 4, 2, P(FAKE), None) == SHAPE
+    assert f(P(FAKE), 4, 0, 2, P(FAKE), None) == SHAPE
+    assert f(P(FAKE), 4, 4, 4, P(FAKE), None) == UNSUP
+    assert f(P(FAKE + 4), 4, 4, 2, P(FAKE), None) == ALIGN
+    assert f(P(FAKE), 4, 4, 2, P(FAKE + 4), None) == ALIGN
+    g = lib.rabit_grad_x
+    need = lib.rabit_gemm_workspace_bytes(16, 8, 2, 8)      # the transposed layer: K x N
+    assert need > 0
+    assert g(None, P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 8, P(FAKE), 16, P(FAKE), need, None) == INVALID
+    assert g(P(FAKE), P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 7, P(FAKE), 16, P(FAKE), need, None) == SHAPE  # ldd < N
+    assert g(P(FAKE), P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 8, P(FAKE), 15, P(FAKE), need, None) == SHAPE  # ldg < K
+    assert g(P(FAKE), P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 8, P(FAKE), 16, P(FAKE), need - 1, None) == WS

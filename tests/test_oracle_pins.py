@@ -405,3 +405,50 @@ def test_scale_grads_hand_case():
     ga, gb = oracle.scale_grads(G, S, a, b)
     assert ga[0, 0] == 7 * 3 - 11 * 5              # -34
     np.testing.assert_array_equal(gb[0], [7 * 2, -11 * 2])
+
+
+def test_grad_x_matches_finite_differences_of_the_layer():
+    # L(x) = sum_{m,n} dY[m][n] * y[m][n] is linear in every x[m][j], so a unit step of the
+    # pinned layer gives dL/dx[m][j] exactly up to float64 rounding.
+    for P in (2, 3):
+        N, K, M = 13, 70, 4
+        W, a, b = _three_path_layer(93, N, K) if P == 3 else (None, None, None)
+        if P == 2:
+            rng0 = np.random.default_rng(92)
+            W = rng0.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)
+            a, b = inputs.scales(92, W)
+        S = oracle.derive_signs(W, a, b, P=P)
+        rng = np.random.default_rng(93 + P)
+        x = rng.standard_normal((M, K))
+        dY = rng.standard_normal((M, N))
+        gx = oracle.grad_x(S, a, b, dY)
+        L = lambda x_: float(np.sum(dY * oracle.layer(S, a, b, x_)))
+        base = L(x)
+        for m, j in [(0, 0), (1, 17), (M - 1, K - 1), (2, 40)]:
+            x2 = x.copy(); x2[m, j] += 1.0
+            assert L(x2) - base == pytest.approx(gx[m, j], rel=1e-9, abs=1e-9), (P, m, j)
+
+
+def test_grad_x_hand_case_and_column_subset():
+    # N=2, K=2, one path: W_hat = [[a0 s00 b0, a0 s01 b1], [a1 s10 b0, a1 s11 b1]]
+    S = np.array([[[1, -1], [-1, -1]]], dtype=np.int8)
+    a = np.array([[2.0, 3.0]]); b = np.array([[5.0, 7.0]])
+    dY = np.array([[1.0, 10.0]])
+    gx = oracle.grad_x(S, a, b, dY)
+    np.testing.assert_array_equal(gx[0], [1 * 2 * 5 - 10 * 3 * 5, -1 * 2 * 7 - 10 * 3 * 7])
+    # the column path: signs and b of columns (1,) only
+    g1 = oracle.grad_x(S[:, :, [1]], a, b, dY, cols=np.array([1]))
+    assert g1[0, 0] == gx[0, 1]
+
+
+def test_grad_x_is_the_transposed_layer():
+    # W_hat^T = sum_k b_k S_k^T a_k: the layer of the transposed signs with a and b exchanged
+    N, K, M = 9, 45, 3
+    rng = np.random.default_rng(95)
+    W = rng.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)
+    a, b = inputs.scales(95, W)
+    S = oracle.derive_signs(W, a, b)
+    dY = rng.standard_normal((M, N))
+    np.testing.assert_allclose(oracle.grad_x(S, a, b, dY),
+                               oracle.layer(np.ascontiguousarray(S.transpose(0, 2, 1)), b, a, dY),
+                               rtol=1e-12, atol=1e-12)
