@@ -519,20 +519,51 @@ def bench_qat_step(rabit, device, hbm_peak, tf_peak, tf_sustained):
         rabit.rabit_derive_pack(Wt, at, bt, packed)
         rabit.rabit_gemm(packed, at, bt, N, K, x, y, ws)
 
+    # backward of the input: the transposed planes, then the GEMM of the transposed layer
+    packed_t = rabit.alloc_packed(K, N, device=device)
+    dy = bf16_tensor(inputs.activations(seed + 1, M, N), device)
+    gx = torch.empty((M, K), device=device)
+    ws_t = rabit.alloc_gemm_workspace(K, N, 2, M, device=device)
+
+    def transpose():
+        rabit.rabit_transpose_pack(packed, N, K, packed_t)
+
+    def grad_x():
+        rabit.rabit_grad_x(packed_t, at, bt, N, K, dy, gx, ws_t)
+
+    derive()
     g_derive = capture_graph(derive)
     g_step = capture_graph(step)
+    g_t = capture_graph(transpose)
+    g_gx = capture_graph(grad_x)
     steps = 20
     ms_d = timed_replays([g_derive], steps, 5, None, device)
     ms_s = timed_replays([g_step], steps, 3, None, device)
+    ms_t = timed_replays([g_t], steps, 5, None, device)
+    ms_g = timed_replays([g_gx], steps, 3, None, device)
     d_bytes = N * K * 4 + 2 * N * K // 8 + 4 * 2 * (N + K)
     gbs = d_bytes * steps / (ms_d * 1e-3) / 1e9
     flops = 2 * 2 * M * N * K
+    t_bytes = 2 * (2 * N * (((K + 127) // 128) * 128) // 8)          # read and write of two planes
+    t_gbs = t_bytes * steps / (ms_t * 1e-3) / 1e9
+    gx_tflops = flops * steps / (ms_g * 1e-3) / 1e12
     return {"derive_pack": {"workload": "llama3_70b_mlp_w_fp32_28672x8192", "value": round(gbs, 1),
                             "unit": "GB/s", "us_per_call": round(ms_d / steps * 1e3, 2),
                             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak,
                                          "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}},
             "qat_step": {"workload": "llama3_70b_mlp_qat_m4096", "ms_per_step": round(ms_s / steps, 4),
-                         "derive_plus_gemm_tflops": round(flops / (ms_s / steps * 1e-3) / 1e12, 1)}}
+                         "derive_plus_gemm_tflops": round(flops / (ms_s / steps * 1e-3) / 1e12, 1)},
+            "qat_backward_x": {"workload": "llama3_70b_mlp_qat_m4096 input gradient",
+                               "transpose_pack": {"us_per_call": round(ms_t / steps * 1e3, 2),
+                                                  "value": round(t_gbs, 1), "unit": "GB/s",
+                                                  "roofline": {"bound": "hbm", "achieved": round(t_gbs, 1),
+                                                               "peak": hbm_peak, "unit": "GB/s",
+                                                               "frac": round(t_gbs / hbm_peak, 4)}},
+                               "grad_x": {"ms_per_call": round(ms_g / steps, 4), "value": round(gx_tflops, 1),
+                                          "unit": "TFLOP/s",
+                                          "roofline": {"bound": "tensor", "achieved": round(gx_tflops, 1),
+                                                       "peak": tf_peak, "unit": "TFLOP/s",
+                                                       "frac": round(gx_tflops / tf_peak, 4)}}}}
 
 
 def cpu_baseline(layers, batch, budget_s=12.0):

@@ -64,14 +64,20 @@ class RowShard:
             rabit.rabit_derive_pack(W_rows, self.a, b, self.packed, P=self.P)
         return self
 
+    def local(self, x: torch.Tensor) -> torch.Tensor:
+        """This rank's outputs, [batch][max_rows] fp32 (columns past its rows are zero)."""
+        batch = x.shape[0]
+        local = torch.zeros((batch, self.max_rows), dtype=torch.float32, device=x.device)
+        if self.rows:
+            rabit.rabit_gemv(self.packed, self.a, self.b, self.rows, self.K, x, local[:, :self.rows], P=self.P)
+        return local
+
     def gemv(self, x: torch.Tensor, y: torch.Tensor, group=None) -> torch.Tensor:
         """y[:, n] for all n of the layer, from this rank's rows and one all-gather.
         Every rank of the group must call it (ranks without rows still join the gather)."""
         import torch.distributed as dist
         batch = x.shape[0]
-        local = torch.zeros((batch, self.max_rows), dtype=torch.float32, device=y.device)
-        if self.rows:
-            rabit.rabit_gemv(self.packed, self.a, self.b, self.rows, self.K, x, local[:, :self.rows], P=self.P)
+        local = self.local(x)
         # ranks' blocks concatenated along dim 0, the form every backend accepts
         gathered = torch.empty((self.world * batch, self.max_rows), dtype=torch.float32, device=y.device)
         dist.all_gather_into_tensor(gathered, local, group=group)
