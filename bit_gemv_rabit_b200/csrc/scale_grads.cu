@@ -152,41 +152,54 @@ scale_grads_tile_kernel(const float *__restrict__ G, int ldg, const uint32_t *__
     }
 }
 
-// The same pass with G staged by TMA: a producer warp keeps kStages boxes of 32 rows x 256
-// columns (32 KiB of fp32) in flight, so the memory parallelism does not depend on registers;
-// eight consumer warps take four rows of each box, reading G from shared memory, and load the
-// next box's sign words and a while the current box is summed.  CTA = one 256-column tile x
-// kBoxesPerCta boxes of rows.  Every wait is bounded: an expired wait sets a fault bit, the
-// consumers contribute zeros, and the producer lets its issued copies land before exiting.
+// The same pass with G staged by TMA, persistent: one CTA per SM walks its share of the
+// tiles (256 rows x 256 columns, eight boxes of 32 rows), and a producer warp keeps kStages
+// stages in flight across tile boundaries, so the stream never drains between tiles.  A stage
+// holds one box of G (32 rows x 256 columns, 32 KiB of fp32), the sign words of the same rows
+// and columns and the rows' a, all brought by TMA, so the consumers read shared memory only.
+// Eight consumer warps take four rows of each box; at a tile's end they add their column
+// sums in shared memory, in a fixed order.  Every wait is
+// bounded: an expired wait sets a fault bit and a flag in shared memory, the consumers stop
+// together at the end of the tile, and the producer lets its issued copies land before exiting.
 constexpr int kBoxRows = 32;
 constexpr int kBoxCols = 256;
 constexpr int kBoxBytes = kBoxRows * kBoxCols * 4;
-constexpr int kStages = 3;
-constexpr int kBoxesPerCta = 8;                  // 256 rows
+constexpr int kStages = 5;
+constexpr int kBoxesPerTile = 8;                 // 256 rows
 constexpr int kTmaThreads = 288;                 // 8 consumer warps + 1 producer warp
-constexpr int kTmaSmem = kStages * kBoxBytes + 128;
+constexpr int kWordsBytesMax = kBoxRows * 32 * 4;             // sign words of a box (P = 3: 32 words a row)
+constexpr int kABytes = 1024;                                 // a of a box's rows (P x 32 floats), padded
+constexpr int kStageBytes = kBoxBytes + kWordsBytesMax + kABytes;
+constexpr int kTmaSmem = kStages * kStageBytes + 128;
 
 template <int kP>
-__global__ void __launch_bounds__(kTmaThreads)
-scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_t *__restrict__ packed,
-                       const float *__restrict__ a, const float *__restrict__ b, int N, int K, int Wr,
+__global__ void __launch_bounds__(kTmaThreads, 1)
+scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_a,
+                       const float *__restrict__ b, int N, int K, int Wr,
                        float *__restrict__ ws_a, float *__restrict__ ws_b, uint32_t *fault,
                        uint64_t timeout_ns, int debug) {
     constexpr int kG = kP == 2 ? 2 : 4;
     constexpr int kSteps = kBoxCols / 128;
     constexpr int kRowsPerWarp = kBoxRows / 8;
+    constexpr int kRowWords = (kBoxCols / 32) * kG;                 // sign words of a box row
+    constexpr uint32_t kTx = kBoxBytes + kBoxRows * kRowWords * 4 + kP * kBoxRows * 4;
     extern __shared__ __align__(128) uint8_t smem[];
-    float *stage = reinterpret_cast<float *>(smem);                       // [kStages][32][256]
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kBoxBytes);
+    // stage s: G [32][256] fp32, then the sign words [32][kRowWords], then a [kP][32]
+    auto stage_g = [&](int st) { return reinterpret_cast<float *>(smem + st * kStageBytes); };
+    auto stage_w = [&](int st) { return reinterpret_cast<const uint32_t *>(smem + st * kStageBytes + kBoxBytes); };
+    auto stage_a = [&](int st) {
+        return reinterpret_cast<const float *>(smem + st * kStageBytes + kBoxBytes + kWordsBytesMax);
+    };
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
     uint64_t *empty = full + kStages;
     __shared__ float colsum[8][kP][kBoxCols];
+    __shared__ int s_abort;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nct = (K + kBoxCols - 1) / kBoxCols;
-    const int ct = blockIdx.x % nct, rb = blockIdx.x / nct;
-    const int c0 = ct * kBoxCols;
-    const int row0 = rb * kBoxRows * kBoxesPerCta;
-    const int boxes = min(kBoxesPerCta, (N - row0 + kBoxRows - 1) / kBoxRows);
+    const int nrb = (N + kBoxRows * kBoxesPerTile - 1) / (kBoxRows * kBoxesPerTile);
+    const int ntiles = nct * nrb;
     int abort_flag = 0;
 
     if (threadIdx.x == 0) {
@@ -194,8 +207,11 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 8);
         }
+        s_abort = 0;
         fence_mbarrier_init();
         prefetch_tensormap(&tmap_g);
+        prefetch_tensormap(&tmap_w);
+        prefetch_tensormap(&tmap_a);
     }
     __syncthreads();
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -204,124 +220,137 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const uint32_
     if (warp == 8) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < boxes; ++c) {
-                const int s = c % kStages;
-                if (!mbar_wait_bounded(smem_u32(&empty[s]), ((c / kStages) & 1) ^ 1, &abort_flag, timeout_ns,
-                                       fault, FAULT_SCALE_GRADS_WAIT))
-                    break;
-                if ((debug & 1) && c == 0) continue;   // fault injection: this box never comes
-                mbar_arrive_expect_tx(smem_u32(&full[s]), kBoxBytes);
-                tma_load_2d(smem_u32(stage + s * kBoxRows * kBoxCols), &tmap_g, smem_u32(&full[s]), c0,
-                            row0 + c * kBoxRows);
-                issued = c + 1;
+            bool issued[kStages] = {};
+            uint32_t last_parity[kStages] = {};
+            bool ok = true;
+            int q = 0;                                 // boxes of this CTA so far (ring position)
+            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+                const int ct = t % nct, rb = t / nct;
+                const int row0 = rb * kBoxRows * kBoxesPerTile;
+                const int boxes = min(kBoxesPerTile, (N - row0 + kBoxRows - 1) / kBoxRows);
+                for (int c = 0; c < boxes; ++c, ++q) {
+                    const int s = q % kStages;
+                    const uint32_t par = static_cast<uint32_t>(q / kStages) & 1u;
+                    if (!mbar_wait_bounded(smem_u32(&empty[s]), par ^ 1u, &abort_flag, timeout_ns, fault,
+                                           FAULT_SCALE_GRADS_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    if ((debug & 1) && q == 0) continue;   // fault injection: this box never comes
+                    const uint32_t bar = smem_u32(&full[s]);
+                    mbar_arrive_expect_tx(bar, kTx);
+                    tma_load_2d(smem_u32(stage_g(s)), &tmap_g, bar, ct * kBoxCols, row0 + c * kBoxRows);
+                    tma_load_2d(smem_u32(stage_w(s)), &tmap_w, bar, ct * kRowWords, row0 + c * kBoxRows);
+                    tma_load_2d(smem_u32(stage_a(s)), &tmap_a, bar, row0 + c * kBoxRows, 0);
+                    issued[s] = true;
+                    last_parity[s] = par;
+                }
             }
-            // Let every issued copy land before the CTA can exit (the consumers stop early on an
+            // Every issued copy lands before the CTA can exit (the consumers stop early on an
             // expired wait).  These are the latest phases of their stages, already complete in
             // normal operation.
             int drain_abort = 0;
-            for (int c = max(0, issued - kStages); c < issued; ++c)
-                if (!((debug & 1) && c == 0))
-                    mbar_wait_bounded(smem_u32(&full[c % kStages]), (c / kStages) & 1, &drain_abort, timeout_ns,
-                                      fault, FAULT_SCALE_GRADS_WAIT);
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s])
+                    mbar_wait_bounded(smem_u32(&full[s]), last_parity[s], &drain_abort, timeout_ns, fault,
+                                      FAULT_SCALE_GRADS_WAIT);
         }
         return;
     }
 
     // ---------------------------------------------------------------- consumers
     // lane's columns: c0 + 128 st + 4 lane + t; group c0/32 + 4 st + lane/8, bits 4(lane%8) + t
-    float bcol[kP][kSteps][4], cacc[kP][kSteps][4];
-#pragma unroll
-    for (int st = 0; st < kSteps; ++st)
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int j = c0 + 128 * st + 4 * lane + t;
-#pragma unroll
-            for (int k = 0; k < kP; ++k) {
-                bcol[k][st][t] = j < K ? __ldg(b + static_cast<int64_t>(k) * K + j) : 0.0f;
-                cacc[k][st][t] = 0.0f;
-            }
-        }
-    struct Side { uint32_t w[kRowsPerWarp][kSteps][kP]; float a[kRowsPerWarp][kP]; };
-    auto load_side = [&](int c, Side &sd) {
-#pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) {
-            const int n = row0 + c * kBoxRows + warp * kRowsPerWarp + i;
-            const bool nok = n < N;
-#pragma unroll
-            for (int st = 0; st < kSteps; ++st) {
-                const int grp = c0 / 32 + 4 * st + (lane >> 3);
-#pragma unroll
-                for (int k = 0; k < kP; ++k)
-                    sd.w[i][st][k] = nok && grp < Wr ? __ldg(packed + (static_cast<int64_t>(n) * Wr + grp) * kG + k) : 0u;
-            }
-#pragma unroll
-            for (int k = 0; k < kP; ++k) sd.a[i][k] = nok ? __ldg(a + static_cast<int64_t>(k) * N + n) : 0.0f;
-        }
-    };
-    Side cur, nxt;
-    load_side(0, nxt);
     const uint32_t sh = 4 * (lane & 7);
-    for (int c = 0; c < boxes; ++c) {
-        cur = nxt;
-        if (c + 1 < boxes) load_side(c + 1, nxt);
-        const int s = c % kStages;
-        const bool ok = mbar_wait_bounded(smem_u32(&full[s]), (c / kStages) & 1, &abort_flag, timeout_ns, fault,
-                                          FAULT_SCALE_GRADS_WAIT);
-        // An expired wait ends this warp's boxes: it stops releasing stages, so the producer's
-        // own bounded wait expires and it drains the copies it issued before the CTA exits.
-        if (!__all_sync(0xffffffffu, ok)) break;
-        const float *box = stage + s * kBoxRows * kBoxCols;
-#pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) {
-            const int r = warp * kRowsPerWarp + i;
-            const int n = row0 + c * kBoxRows + r;
-            float racc[kP];
-#pragma unroll
-            for (int k = 0; k < kP; ++k) racc[k] = 0.0f;
-#pragma unroll
-            for (int st = 0; st < kSteps; ++st) {
-                const float4 g4 = *reinterpret_cast<const float4 *>(box + r * kBoxCols + 128 * st + 4 * lane);
-                const float gvals[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-                for (int k = 0; k < kP; ++k) {
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        // s = +1 for bit 0, -1 for bit 1: flip the sign bit of G
-                        const float gs = __uint_as_float(__float_as_uint(gvals[t]) ^
-                                                         (((cur.w[i][st][k] >> (sh + t)) & 1u) << 31));
-                        racc[k] = fmaf(gs, bcol[k][st][t], racc[k]);
-                        cacc[k][st][t] = fmaf(gs, cur.a[i][k], cacc[k][st][t]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < kP; ++k) {
-                float v = racc[k];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0 && n < N) ws_a[(static_cast<int64_t>(k) * nct + ct) * N + n] = v;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-    }
-    // column sums of the tile: over the 8 consumer warps, in a fixed order
-#pragma unroll
-    for (int k = 0; k < kP; ++k)
+    int q = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int ct = t % nct, rb = t / nct;
+        const int c0 = ct * kBoxCols;
+        const int row0 = rb * kBoxRows * kBoxesPerTile;
+        const int boxes = min(kBoxesPerTile, (N - row0 + kBoxRows - 1) / kBoxRows);
+        float bcol[kP][kSteps][4], cacc[kP][kSteps][4];
 #pragma unroll
         for (int st = 0; st < kSteps; ++st)
 #pragma unroll
-            for (int t = 0; t < 4; ++t) colsum[warp][k][128 * st + 4 * lane + t] = cacc[k][st][t];
-    asm volatile("bar.sync 1, 256;" ::: "memory");   // the 8 consumer warps only
-    const int nrb = (N + kBoxRows * kBoxesPerCta - 1) / (kBoxRows * kBoxesPerCta);
-    for (int u = threadIdx.x; u < kP * kBoxCols; u += 256) {
-        const int k = u / kBoxCols, cc = u % kBoxCols;
-        const int j = c0 + cc;
-        if (j >= K) continue;
-        float v = 0.0f;
-        for (int w = 0; w < 8; ++w) v += colsum[w][k][cc];
-        ws_b[(static_cast<int64_t>(k) * nrb + rb) * K + j] = v;
+            for (int tt = 0; tt < 4; ++tt) {
+                const int j = c0 + 128 * st + 4 * lane + tt;
+#pragma unroll
+                for (int k = 0; k < kP; ++k) {
+                    bcol[k][st][tt] = j < K ? __ldg(b + static_cast<int64_t>(k) * K + j) : 0.0f;
+                    cacc[k][st][tt] = 0.0f;
+                }
+            }
+        for (int c = 0; c < boxes; ++c, ++q) {
+            const int s = q % kStages;
+            const bool ok = mbar_wait_bounded(smem_u32(&full[s]), static_cast<uint32_t>(q / kStages) & 1u,
+                                              &abort_flag, timeout_ns, fault, FAULT_SCALE_GRADS_WAIT);
+            // An expired wait ends this warp's boxes: it stops releasing stages, so the producer's
+            // own bounded wait expires and it drains the copies it issued before the CTA exits;
+            // the flag stops every consumer warp at the end of this tile.
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) s_abort = 1;
+                break;
+            }
+            const uint32_t *words = stage_w(s);
+            const float *arow = stage_a(s);
+            const float *box = stage_g(s);
+#pragma unroll
+            for (int i = 0; i < kRowsPerWarp; ++i) {
+                const int r = warp * kRowsPerWarp + i;
+                const int n = row0 + c * kBoxRows + r;
+                float racc[kP], av[kP];
+                uint32_t wv[kSteps][kP];
+#pragma unroll
+                for (int k = 0; k < kP; ++k) {
+                    racc[k] = 0.0f;
+                    av[k] = arow[k * kBoxRows + r];
+#pragma unroll
+                    for (int st = 0; st < kSteps; ++st) wv[st][k] = words[r * kRowWords + (4 * st + (lane >> 3)) * kG + k];
+                }
+#pragma unroll
+                for (int st = 0; st < kSteps; ++st) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(box + r * kBoxCols + 128 * st + 4 * lane);
+                    const float gvals[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                    for (int k = 0; k < kP; ++k) {
+#pragma unroll
+                        for (int tt = 0; tt < 4; ++tt) {
+                            // s = +1 for bit 0, -1 for bit 1: flip the sign bit of G
+                            const float gs = __uint_as_float(__float_as_uint(gvals[tt]) ^
+                                                             (((wv[st][k] >> (sh + tt)) & 1u) << 31));
+                            racc[k] = fmaf(gs, bcol[k][st][tt], racc[k]);
+                            cacc[k][st][tt] = fmaf(gs, av[k], cacc[k][st][tt]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < kP; ++k) {
+                    float v = racc[k];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if (lane == 0 && n < N) ws_a[(static_cast<int64_t>(k) * nct + ct) * N + n] = v;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+        }
+        // column sums of the tile: over the 8 consumer warps, in a fixed order
+#pragma unroll
+        for (int k = 0; k < kP; ++k)
+#pragma unroll
+            for (int st = 0; st < kSteps; ++st)
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) colsum[warp][k][128 * st + 4 * lane + tt] = cacc[k][st][tt];
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // the 8 consumer warps only
+        for (int u = threadIdx.x; u < kP * kBoxCols; u += 256) {
+            const int k = u / kBoxCols, cc = u % kBoxCols;
+            const int j = c0 + cc;
+            if (j >= K) continue;
+            float v = 0.0f;
+            for (int w = 0; w < 8; ++w) v += colsum[w][k][cc];
+            ws_b[(static_cast<int64_t>(k) * nrb + rb) * K + j] = v;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // colsum is rewritten by the next tile
+        if (s_abort) break;                              // every consumer warp sees the same flag here
     }
 }
 
@@ -384,9 +413,11 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
     cfg.numAttrs = 1;
     int nrb = 0;
     cudaError_t e = cudaSuccess;
-    // TMA-staged pass when the tensor map can describe G (16-byte aligned base and pitch).
+    // TMA-staged pass when tensor maps can describe G (16-byte aligned base and pitch) and a.
     auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
-    const bool tma = encode && (reinterpret_cast<uintptr_t>(G) % 16 == 0) && ((static_cast<int64_t>(ldg) * 4) % 16 == 0);
+    // (a is staged by TMA as well: 16-byte aligned base and rows of N floats, N a multiple of 4)
+    const bool tma = encode && (reinterpret_cast<uintptr_t>(G) % 16 == 0) && ((static_cast<int64_t>(ldg) * 4) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(a) % 16 == 0) && (N % 4 == 0);
     if (tma) {
         CUtensorMap tmap;
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
@@ -397,16 +428,33 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
                             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        // the sign words of a box: kRowWords words of each of its rows; a of its rows, per path
+        const int G = P == 2 ? 2 : 4;
+        CUtensorMap tmap_w, tmap_a;
+        cuuint64_t wdims[2] = {static_cast<cuuint64_t>(Wr) * G, static_cast<cuuint64_t>(N)};
+        cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(Wr) * G * 4};
+        cuuint32_t wbox[2] = {static_cast<cuuint32_t>((kBoxCols / 32) * G), kBoxRows};
+        r = encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(packed), wdims, wstrides, wbox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        cuuint64_t adims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(P)};
+        cuuint64_t astrides[1] = {static_cast<cuuint64_t>(N) * 4};
+        cuuint32_t abox[2] = {kBoxRows, static_cast<cuuint32_t>(P)};
+        r = encode(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(a), adims, astrides, abox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
         static ContextFlags opted[2];
-        void (*kern)(CUtensorMap, const uint32_t *, const float *, const float *, int, int, int, float *, float *,
+        void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, const float *, int, int, int, float *, float *,
                      uint32_t *, uint64_t, int) = P == 2 ? scale_grads_tma_kernel<2> : scale_grads_tma_kernel<3>;
         e = ensure_smem_optin(ctx, kern, kTmaSmem, opted[P - 2]);
         if (e != cudaSuccess) return e;
-        nrb = (N + kBoxRows * kBoxesPerCta - 1) / (kBoxRows * kBoxesPerCta);
-        cfg.gridDim = dim3(static_cast<unsigned>(nct) * static_cast<unsigned>(nrb));
+        nrb = (N + kBoxRows * kBoxesPerTile - 1) / (kBoxRows * kBoxesPerTile);
+        cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(nct) * nrb, ctx.num_sms)));
         cfg.blockDim = dim3(kTmaThreads);
         cfg.dynamicSmemBytes = kTmaSmem;
-        e = cudaLaunchKernelEx(&cfg, kern, tmap, packed, a, b, N, K, Wr, ws_a, ws_b, fault_word, timeout_ns,
+        e = cudaLaunchKernelEx(&cfg, kern, tmap, tmap_w, tmap_a, b, N, K, Wr, ws_a, ws_b, fault_word, timeout_ns,
                                debug);
     } else {
         nrb = (N + kTileRows - 1) / kTileRows;
