@@ -9,6 +9,12 @@
 // with both paths concatenated along the contraction dimension (64-column blocks of path 1
 // and path 2 alternate), so one fp32 accumulator holds the whole output tile.
 //
+// One launch serves one layer or a group of up to four independent layers with the same
+// token count (e.g. the gate and up projections of an MLP): their tiles share the persistent
+// CTAs.  Tiles of a long contraction cost more, so the host deals them longest first, each
+// to the least loaded CTA, and passes every CTA's list in the kernel arguments; all roles of
+// a CTA walk the same list.
+//
 // Kernel structure (one persistent CTA per SM, 6 warps):
 //   warp 0      TMA producer: X' tiles (256 tokens x 64 columns, 128-byte swizzle) into a
 //               4-stage shared-memory ring.
@@ -33,6 +39,11 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <mutex>
+#include <queue>
+#include <vector>
+
 #include "rabit.h"
 #include "rabit_device.cuh"
 #include "rabit_kernels.h"
@@ -51,15 +62,32 @@ constexpr uint32_t kAccCol = 0;      // accumulator: columns [0, 256)
 constexpr uint32_t kACol = 256;      // A stages: columns [256 + 32 s, 256 + 32 s + 32)
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 
-struct GemmArgs {
+constexpr int kMaxGemmGroup = 4;
+constexpr int kMaxGrid = 160;
+constexpr int kMaxListedTiles = 6144;   // tiles a launch may list (kernel-parameter space)
+
+struct GemmProb {
     const uint32_t *packed;
     const float *a;
     float *y;
+    int N, K, Kp, ldy;
+    int tiles_m;             // token tiles
+    int tile0;               // the layer's first tile in the launch
+};
+
+struct GemmMaps {
+    CUtensorMap x[kMaxGemmGroup];   // X' of each layer: [P][M][Kp] fp16
+};
+
+struct GemmArgs {
+    GemmProb prob[kMaxGemmGroup];
     uint32_t *fault;
     uint64_t timeout_ns;
-    int N, K, M, Kp, ldy;
-    int tiles_m, num_tiles;
+    int nprob, M, num_tiles;
     int debug;
+    int listed;              // 1: CTA c takes order[begin[c] .. begin[c+1]); 0: tiles c, c + grid, ...
+    uint16_t begin[kMaxGrid + 1];
+    uint16_t order[kMaxListedTiles];
 };
 
 struct SmemCtl {
@@ -77,17 +105,30 @@ __device__ __forceinline__ uint32_t half_bits(float v) {
     return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v)));
 }
 
+// The CTA's i-th tile, and the layer it belongs to.
+__device__ __forceinline__ int cta_tile(const GemmArgs &p, int i) {
+    return p.listed ? static_cast<int>(p.order[p.begin[blockIdx.x] + i]) : static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+}
+__device__ __forceinline__ int cta_tile_count(const GemmArgs &p) {
+    return p.listed ? p.begin[blockIdx.x + 1] - p.begin[blockIdx.x]
+                    : (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+}
+__device__ __forceinline__ int prob_of_tile(const GemmArgs &p, int tile) {
+    int l = 0;
+    while (l + 1 < p.nprob && tile >= p.prob[l + 1].tile0) ++l;
+    return l;
+}
+
 template <int kP>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
+gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + kStages * kStageBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kblocks_per_path = p.Kp / kBK;
-    const int nkb = kP * kblocks_per_path;
+    const int ntiles = cta_tile_count(p);
     volatile int *abort_flag = &ctl->abort;
 
     if (threadIdx.x == 0) {
@@ -101,7 +142,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
         mbar_init(smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
         fence_mbarrier_init();
-        prefetch_tensormap(&tmap_x);
+        for (int l = 0; l < p.nprob; ++l) prefetch_tensormap(&maps.x[l]);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&ctl->tmem_base), kTmemCols);
@@ -123,8 +164,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
             uint32_t last_parity[kStages];
             bool issued[kStages];
             for (int s = 0; s < kStages; ++s) issued[s] = false;
-            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-                const int m0 = (tile % p.tiles_m) * kBN;
+            for (int ti = 0; ok && ti < ntiles; ++ti) {
+                const int tile = cta_tile(p, ti);
+                const int l = prob_of_tile(p, tile);
+                const GemmProb &q = p.prob[l];
+                const int m0 = ((tile - q.tile0) % q.tiles_m) * kBN;
+                const int nkb = kP * (q.Kp / kBK);
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
                     if (!mbar_wait_bounded(smem_u32(&ctl->empty[s]), ph ^ 1u, abort_flag,
@@ -136,7 +181,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
                     mbar_arrive_expect_tx(bar, kStageBytes);
                     const int path = kb % kP;           // K blocks cycle through the paths
                     const int kcol = (kb / kP) * kBK;
-                    tma_load_3d(smem_u32(smem + s * kStageBytes), &tmap_x, bar, kcol, m0, path);
+                    tma_load_3d(smem_u32(smem + s * kStageBytes), &maps.x[l], bar, kcol, m0, path);
                     issued[s] = true;
                     last_parity[s] = ph;
                 }
@@ -159,7 +204,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
             uint32_t it = 0, local_tile = 0;
             bool ok = true;
             bool any_issued = false;
-            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local_tile) {
+            for (int ti = 0; ok && ti < ntiles; ++ti, ++local_tile) {
+                const int nkb = kP * (p.prob[prob_of_tile(p, cta_tile(p, ti))].Kp / kBK);
                 if (!mbar_wait_bounded(smem_u32(&ctl->acc_empty), (local_tile & 1u) ^ 1u, abort_flag,
                                        p.timeout_ns, p.fault, FAULT_GEMM_WAIT_EPILOGUE)) {
                     ok = false;
@@ -202,18 +248,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;          // row within the tile == TMEM lane
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        const int Wr = p.Kp / 32;               // 32-column groups per row
         uint32_t it = 0, local_tile = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local_tile) {
-            const int m0 = (tile % p.tiles_m) * kBN;
-            const int n0 = (tile / p.tiles_m) * kBM;
+        for (int ti = 0; ok && ti < ntiles; ++ti, ++local_tile) {
+            const int tile = cta_tile(p, ti);
+            const GemmProb &q = p.prob[prob_of_tile(p, tile)];
+            const int Wr = q.Kp / 32;               // 32-column groups per row
+            const int kblocks_per_path = q.Kp / kBK;
+            const int nkb = kP * kblocks_per_path;
+            const int m0 = ((tile - q.tile0) % q.tiles_m) * kBN;
+            const int n0 = ((tile - q.tile0) / q.tiles_m) * kBM;
             const int n = n0 + row;
-            const bool row_valid = n < p.N;
+            const bool row_valid = n < q.N;
             uint32_t a2[kP];
 #pragma unroll
             for (int k = 0; k < kP; ++k) {
-                const uint32_t h = row_valid ? half_bits(__ldg(p.a + k * p.N + n)) : 0u;
+                const uint32_t h = row_valid ? half_bits(__ldg(q.a + k * q.N + n)) : 0u;
                 a2[k] = h | (h << 16);
             }
             // The packed words of one 64-column block (two 32-column groups) of this row:
@@ -221,7 +271,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
             // three paths: two 16-byte loads {path1, path2, path3, pad} of groups w and w+1.
             struct Block { uint4 g0, g1; };
             constexpr int kGroupWords = kP == 2 ? 2 : 4;     // words per 32-column group
-            const uint4 *row_ptr = reinterpret_cast<const uint4 *>(p.packed + static_cast<int64_t>(n) * Wr * kGroupWords);
+            const uint4 *row_ptr = reinterpret_cast<const uint4 *>(q.packed + static_cast<int64_t>(n) * Wr * kGroupWords);
             auto load_block = [&](int blk) -> Block {
                 Block r{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
                 if (row_valid) {
@@ -289,7 +339,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs p) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int m = m0 + c0 + i;
-                        if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __uint_as_float(acc[i]);
+                        if (m < p.M) q.y[static_cast<int64_t>(m) * q.ldy + n] = __uint_as_float(acc[i]);
                     }
                 }
             }
@@ -371,38 +421,109 @@ size_t gemm_workspace_bytes(int N, int K, int P, int M) {
     return static_cast<size_t>(P) * static_cast<size_t>(M) * static_cast<size_t>(padded_cols(K)) * 2;
 }
 
-cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
-                        const float *b, int N, int K, int P, const uint16_t *x, int M, int ldx,
-                        float *y, int ldy, void *workspace, uint32_t *fault_word,
-                        uint64_t timeout_ns, int debug_flags) {
-    if (P != 2 && P != 3) return cudaErrorInvalidValue;
-    const int Kp = static_cast<int>(padded_cols(K));
+namespace {
+inline size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+}  // namespace
 
+size_t gemm_group_workspace_bytes(const GemvLayer *layers, int count, int P, int M) {
+    size_t total = 0;
+    for (int i = 0; i < count; ++i) total += up256(gemm_workspace_bytes(layers[i].N, layers[i].K, P, M));
+    return total;
+}
+
+cudaError_t launch_gemm_group(const LaunchCtx &ctx, const GemvLayer *layers, int count, int P, int M,
+                              void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug_flags) {
+    if ((P != 2 && P != 3) || count < 1 || count > kMaxGemmGroup) return cudaErrorInvalidValue;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = ctx.pdl ? 1 : 0;
 
-    // 1. Tensor map over the workspace viewed as [P][M][Kp] fp16.
+    // 1. Tensor maps over each layer's part of the workspace, viewed as [P][M][Kp] fp16.
     auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
     if (!encode) return cudaErrorNotSupported;
-    CUtensorMap tmap;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(P)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kp) * 2, static_cast<cuuint64_t>(M) * Kp * 2};
-    cuuint32_t box[3] = {kBK, kBN, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, workspace, dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    GemmMaps maps{};
+    static GemmArgs args;               // large (the tile lists); filled and copied per launch
+    static std::mutex args_mutex;
+    std::lock_guard<std::mutex> guard(args_mutex);
+    args = GemmArgs{};
+    uint8_t *xp[kMaxGemmGroup];
+    {
+        size_t off = 0;
+        int tiles = 0;
+        for (int i = 0; i < count; ++i) {
+            const GemvLayer &l = layers[i];
+            const int Kp = static_cast<int>(padded_cols(l.K));
+            xp[i] = static_cast<uint8_t *>(workspace) + off;
+            off += up256(gemm_workspace_bytes(l.N, l.K, P, M));
+            cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kp), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(P)};
+            cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kp) * 2, static_cast<cuuint64_t>(M) * Kp * 2};
+            cuuint32_t box[3] = {kBK, kBN, 1};
+            cuuint32_t estr[3] = {1, 1, 1};
+            CUresult r = encode(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, xp[i], dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+            GemmProb &q = args.prob[i];
+            q.packed = l.packed;
+            q.a = l.a;
+            q.y = l.y;
+            q.N = l.N;
+            q.K = l.K;
+            q.Kp = Kp;
+            q.ldy = l.ldy;
+            q.tiles_m = (M + kBN - 1) / kBN;
+            q.tile0 = tiles;
+            tiles += q.tiles_m * ((l.N + kBM - 1) / kBM);
+        }
+        args.num_tiles = tiles;
+    }
+    args.nprob = count;
+    args.M = M;
+    args.fault = fault_word;
+    args.timeout_ns = timeout_ns;
+    args.debug = debug_flags;
+    const int grid = std::min(args.num_tiles, std::min(ctx.num_sms, kMaxGrid));
 
-    // 2. Shared-memory opt-in.  Steps 1 and 2 can fail, so they come before anything is
+    // 2. The tile lists: longest contraction first, each tile to the least loaded CTA (ties:
+    //    the lowest CTA), so every run deals the same tiles to the same CTAs.
+    args.listed = args.num_tiles <= kMaxListedTiles ? 1 : 0;
+    if (args.listed) {
+        std::vector<int> tiles(args.num_tiles);
+        for (int t = 0; t < args.num_tiles; ++t) tiles[t] = t;
+        auto cost = [&](int t) {
+            int l = 0;
+            while (l + 1 < count && t >= args.prob[l + 1].tile0) ++l;
+            return args.prob[l].Kp;
+        };
+        std::stable_sort(tiles.begin(), tiles.end(), [&](int x, int y) { return cost(x) > cost(y); });
+        std::vector<std::vector<int>> lists(grid);
+        using Slot = std::pair<long long, int>;                       // (load, CTA)
+        std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+        for (int c = 0; c < grid; ++c) heap.push({0, c});
+        for (int t : tiles) {
+            Slot sl = heap.top();
+            heap.pop();
+            lists[sl.second].push_back(t);
+            heap.push({sl.first + cost(t), sl.second});
+        }
+        int pos = 0;
+        for (int c = 0; c < grid; ++c) {
+            args.begin[c] = static_cast<uint16_t>(pos);
+            for (int t : lists[c]) args.order[pos++] = static_cast<uint16_t>(t);
+        }
+        args.begin[grid] = static_cast<uint16_t>(pos);
+    }
+
+    // 3. Shared-memory opt-in.  Steps 1 to 3 can fail, so they come before anything is
     //    enqueued: a call that returns an error has put no work on the stream.
-    void (*kern)(CUtensorMap, GemmArgs) = P == 2 ? gemm_kernel<2> : gemm_kernel<3>;
+    void (*kern)(GemmMaps, GemmArgs) = P == 2 ? gemm_kernel<2> : gemm_kernel<3>;
     static ContextFlags opted[2];
     if (cudaError_t e = ensure_smem_optin(ctx, kern, kSmemBytes, opted[P - 2]); e != cudaSuccess) return e;
 
-    // 3. X'_k = fp16(x (.) b_k), permuted within 32-column groups.
-    {
+    // 4. X'_k = fp16(x (.) b_k) of each layer, permuted within 32-column groups.
+    for (int i = 0; i < count; ++i) {
+        const GemvLayer &l = layers[i];
+        const int Kp = args.prob[i].Kp;
         const int64_t total = static_cast<int64_t>(P) * M * (Kp / 2);
         int64_t blocks = (total + 255) / 256;
         if (blocks > static_cast<int64_t>(ctx.num_sms) * 16) blocks = static_cast<int64_t>(ctx.num_sms) * 16;
@@ -412,29 +533,12 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
         cfg.stream = ctx.stream;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, prep_x_kernel, x, ldx, b, K, Kp, M, P,
-                                           static_cast<uint32_t *>(workspace));
+        cudaError_t e = cudaLaunchKernelEx(&cfg, prep_x_kernel, static_cast<const uint16_t *>(l.x), l.ldx, l.b, l.K,
+                                           Kp, M, P, reinterpret_cast<uint32_t *>(xp[i]));
         if (e != cudaSuccess) return e;
     }
 
-    // 4. Persistent tcgen05 kernel.
-    GemmArgs args;
-    args.packed = packed;
-    args.a = a;
-    args.y = y;
-    args.fault = fault_word;
-    args.timeout_ns = timeout_ns;
-    args.N = N;
-    args.K = K;
-    args.M = M;
-    args.Kp = Kp;
-    args.ldy = ldy;
-    args.tiles_m = (M + kBN - 1) / kBN;
-    const int tiles_n = (N + kBM - 1) / kBM;
-    args.num_tiles = args.tiles_m * tiles_n;
-    args.debug = debug_flags;
-
-    int grid = args.num_tiles < ctx.num_sms ? args.num_tiles : ctx.num_sms;
+    // 5. Persistent tcgen05 kernel.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kThreads);
@@ -442,7 +546,15 @@ cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const floa
     cfg.stream = ctx.stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmap, args);
+    return cudaLaunchKernelEx(&cfg, kern, maps, args);
+}
+
+cudaError_t launch_gemm(const LaunchCtx &ctx, const uint32_t *packed, const float *a,
+                        const float *b, int N, int K, int P, const uint16_t *x, int M, int ldx,
+                        float *y, int ldy, void *workspace, uint32_t *fault_word,
+                        uint64_t timeout_ns, int debug_flags) {
+    GemvLayer l{packed, a, b, N, K, x, ldx, y, ldy};
+    return launch_gemm_group(ctx, &l, 1, P, M, workspace, fault_word, timeout_ns, debug_flags);
 }
 
 }  // namespace rabit

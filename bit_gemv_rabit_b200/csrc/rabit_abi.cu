@@ -275,6 +275,42 @@ int rabit_gemm(const uint32_t *packed, const float *a, const float *b, int N, in
                                             workspace, fault, timeout_ns, debug));
 }
 
+size_t rabit_gemm_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count, int P, int M) {
+    if (!layers || count < 1 || count > RABIT_GEMM_MAX_GROUP || (P != 2 && P != 3) || M < 1) return 0;
+    rabit::GemvLayer g[RABIT_GEMM_MAX_GROUP];
+    for (int i = 0; i < count; ++i) {
+        if (layers[i].N < 1 || layers[i].K < 1) return 0;
+        g[i] = rabit::GemvLayer{layers[i].packed, layers[i].a, layers[i].b, layers[i].N, layers[i].K,
+                                layers[i].x, layers[i].ldx, layers[i].y, layers[i].ldy};
+    }
+    return rabit::gemm_group_workspace_bytes(g, count, P, M);
+}
+
+int rabit_gemm_grouped(const rabit_gemv_layer *layers, int count, int P, int M, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+    if (!layers || count < 1 || count > RABIT_GEMM_MAX_GROUP) return RABIT_ERR_INVALID_ARG;
+    if (P < 1 || M < 1) return RABIT_ERR_SHAPE;
+    rabit::GemvLayer g[RABIT_GEMM_MAX_GROUP];
+    for (int i = 0; i < count; ++i) {
+        const rabit_gemv_layer &l = layers[i];
+        if (!l.packed || !l.a || !l.b || !l.x || !l.y) return RABIT_ERR_INVALID_ARG;
+        if (l.N < 1 || l.K < 1 || l.ldx < l.K || l.ldy < l.N) return RABIT_ERR_SHAPE;
+        if (!aligned(l.packed, 16) || !aligned(l.x, 16) || (l.ldx % 8) != 0 || !aligned(l.y, 4))
+            return RABIT_ERR_ALIGNMENT;
+        g[i] = rabit::GemvLayer{l.packed, l.a, l.b, l.N, l.K, l.x, l.ldx, l.y, l.ldy};
+    }
+    if (P != 2 && P != 3) return RABIT_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < rabit::gemm_group_workspace_bytes(g, count, P, M))
+        return RABIT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return RABIT_ERR_ALIGNMENT;
+    rabit::LaunchCtx ctx;
+    uint32_t *fault = nullptr;
+    int st = device_ctx(stream, ctx, &fault);
+    if (st != RABIT_OK) return st;
+    const int debug = env_flag("RABIT_TEST_SKIP_ONE_ARRIVE") ? 1 : 0;
+    return finish_launch(rabit::launch_gemm_group(ctx, g, count, P, M, workspace, fault, wait_timeout_ns(), debug));
+}
+
 int rabit_transpose_pack(const uint32_t *packed, int N, int K, int P, uint32_t *packed_t, void *stream) {
     if (!packed || !packed_t) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || P < 1) return RABIT_ERR_SHAPE;

@@ -88,6 +88,10 @@ cudaError_t launch_svid_init(const LaunchCtx &ctx, const float *W, int ldw, int 
                              uint32_t *fault_word, uint64_t timeout_ns);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
+// Up to 4 layers with the same token count in one launch (gemm.cu); x of each layer is bf16.
+size_t gemm_group_workspace_bytes(const GemvLayer *layers, int count, int P, int M);
+cudaError_t launch_gemm_group(const LaunchCtx &ctx, const GemvLayer *layers, int count, int P, int M,
+                              void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug_flags);
 // Device address (in the launch's context) and size of the library's fixed GEMM scratch
 // buffer (rabit_gemm_noalloc).
 cudaError_t gemm_noalloc_scratch(const LaunchCtx &ctx, void **ptr, size_t *bytes);

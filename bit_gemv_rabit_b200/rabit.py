@@ -32,6 +32,8 @@ SIGNATURES = [
     ("rabit_gemm_workspace_bytes", _sz, [_i, _i, _i, _i]),
     ("rabit_gemm", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_gemm_noalloc", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p]),
+    ("rabit_gemm_grouped_workspace_bytes", _sz, [_p, _i, _i, _i]),
+    ("rabit_gemm_grouped", _i, [_p, _i, _i, _i, _p, _sz, _p]),
     ("rabit_transpose_pack", _i, [_p, _i, _i, _i, _p, _p]),
     ("rabit_grad_x", _i, [_p, _p, _p, _i, _i, _i, _p, _i, _i, _p, _i, _p, _sz, _p]),
     ("rabit_scale_grads_workspace_bytes", _sz, [_i, _i, _i]),
@@ -191,6 +193,28 @@ def rabit_gemm(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K
                              _dptr(y), y.stride(0), _dptr(workspace), ws_bytes, _stream(stream)),
            "rabit_gemm")
     return y
+
+
+def rabit_gemm_grouped_workspace_bytes(layers, P: int = 2) -> int:
+    """layers: sequence of (packed, a, b, N, K, x, y) with x bf16 [M][K] (the same M)."""
+    arr = _layer_array(layers)
+    return int(load().rabit_gemm_grouped_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(layers), P,
+                                                         layers[0][5].shape[0]))
+
+
+def alloc_gemm_grouped_workspace(layers, P: int = 2, device=None) -> torch.Tensor:
+    return torch.empty(rabit_gemm_grouped_workspace_bytes(layers, P), dtype=torch.uint8, device=device or "cuda")
+
+
+def rabit_gemm_grouped(layers, workspace: torch.Tensor, P: int = 2, stream=None):
+    """layers: sequence of (packed, a, b, N, K, x, y); one launch computes rabit_gemm for each."""
+    arr = _layer_array(layers)
+    M = layers[0][5].shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().rabit_gemm_grouped(ctypes.cast(arr, ctypes.c_void_p), len(layers), P, M, _dptr(workspace),
+                                     ws_bytes, _stream(stream)),
+           "rabit_gemm_grouped")
+    return [layer[6] for layer in layers]
 
 
 def rabit_transpose_pack(packed: torch.Tensor, N: int, K: int, packed_t: torch.Tensor, P: int = 2,

@@ -191,6 +191,25 @@ RABIT_API int rabit_gemm(const uint32_t *packed, const float *a, const float *b,
                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * rabit_gemm_grouped -- rabit_gemm for up to RABIT_GEMM_MAX_GROUP independent layers with the
+ * same token count M in one persistent launch (e.g. the gate and up projections of an MLP,
+ * which read the same x).  Each layer computes exactly what rabit_gemm computes for it; the
+ * layers' tiles share the CTAs, dealt longest contraction first to the least loaded CTA, so
+ * the last wave of one layer no longer leaves SMs idle.
+ *   layers     host array of `count` descriptions (struct rabit_gemv_layer): packed, a, b, N,
+ *              K as for rabit_gemm; x = bf16 [M][ldx] (16-byte aligned, ldx >= K and a
+ *              multiple of 8); y = fp32 [M][ldy] (output), ldy >= N
+ *   workspace  at least rabit_gemm_grouped_workspace_bytes(layers, count, P, M) bytes,
+ *              256-byte aligned (0 from the size call means invalid arguments)
+ * Accuracy and errors: those of rabit_gemm, plus INVALID_ARG for a null `layers` or count
+ * out of range.
+ */
+#define RABIT_GEMM_MAX_GROUP 4
+RABIT_API size_t rabit_gemm_grouped_workspace_bytes(const rabit_gemv_layer *layers, int count, int P, int M);
+RABIT_API int rabit_gemm_grouped(const rabit_gemv_layer *layers, int count, int P, int M, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/*
  * rabit_transpose_pack -- the packed sign planes of W^T from those of W, for the input
  * gradient (sec. 4.1: W_hat = sum_k a_k (.) S_k (.) b_k, so W_hat^T = sum_k b_k (.) S_k^T (.) a_k
  * is a stacked layer of the same form, K x N, with a and b exchanged):

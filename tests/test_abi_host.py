@@ -227,3 +227,27 @@ def test_transpose_pack_and_grad_x_validation(lib):
     assert g(P(FAKE), P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 7, P(FAKE), 16, P(FAKE), need, None) == SHAPE  # ldd < N
     assert g(P(FAKE), P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 8, P(FAKE), 15, P(FAKE), need, None) == SHAPE  # ldg < K
     assert g(P(FAKE), P(FAKE), P(FAKE), 8, 16, 2, P(FAKE), 8, 8, P(FAKE), 16, P(FAKE), need - 1, None) == WS
+
+
+def test_gemm_grouped_validation(lib):
+    L = rabit.GemvLayer
+    good = dict(packed=FAKE, a=FAKE, b=FAKE, N=8, K=16, x=FAKE, ldx=16, y=FAKE, ldy=8)
+    def arr(**kw):
+        d = dict(good, **kw)
+        a = (L * 2)(L(**good), L(**d))
+        return ctypes.cast(a, ctypes.c_void_p)
+    need = lib.rabit_gemm_grouped_workspace_bytes(arr(), 2, 2, 8)
+    # each layer's X' ([P][M][Kp] fp16) in its own 256-byte aligned region
+    assert need == 2 * (2 * 8 * 128 * 2)
+    assert lib.rabit_gemm_grouped_workspace_bytes(arr(), 5, 2, 8) == 0
+    assert lib.rabit_gemm_grouped_workspace_bytes(arr(), 2, 4, 8) == 0
+    f = lib.rabit_gemm_grouped
+    assert f(None, 2, 2, 8, P(FAKE), need, None) == INVALID
+    assert f(arr(), 5, 2, 8, P(FAKE), need, None) == INVALID
+    assert f(arr(y=0), 2, 2, 8, P(FAKE), need, None) == INVALID
+    assert f(arr(ldx=8), 2, 2, 8, P(FAKE), need, None) == SHAPE
+    assert f(arr(ldx=20), 2, 2, 8, P(FAKE), need, None) == ALIGN
+    assert f(arr(x=FAKE + 8), 2, 2, 8, P(FAKE), need, None) == ALIGN
+    assert f(arr(), 2, 4, 8, P(FAKE), need, None) == UNSUP
+    assert f(arr(), 2, 2, 8, P(FAKE), need - 1, None) == WS
+    assert f(arr(), 2, 2, 8, P(FAKE + 128), need, None) == ALIGN
