@@ -386,11 +386,12 @@ size_t rabit_svid_init_workspace_bytes(int N, int K, int P) {
     return rabit::svid_workspace_bytes(N, K, P);
 }
 
-int rabit_svid_init(const float *W, int N, int K, int ldw, int P, int T, int power_iters,
+int rabit_svid_init(const float *W, int N, int K, int ldw, int P, int T, int power_iters, float power_tol,
                     const float *s_in, const float *s_out, float alpha_in, float alpha_out, float *a,
                     float *b, uint32_t *packed, void *workspace, size_t workspace_bytes, void *stream) {
     if (!W || !s_in || !s_out || !a || !b || !packed) return RABIT_ERR_INVALID_ARG;
     if (!std::isfinite(alpha_in) || !std::isfinite(alpha_out)) return RABIT_ERR_INVALID_ARG;
+    if (!(power_tol >= 0.0f) || !std::isfinite(power_tol)) return RABIT_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || ldw < K || T < 1 || T > RABIT_SVID_MAX_ITERS || power_iters < 1 ||
         power_iters > RABIT_SVID_MAX_ITERS)
         return RABIT_ERR_SHAPE;
@@ -404,8 +405,9 @@ int rabit_svid_init(const float *W, int N, int K, int ldw, int P, int T, int pow
     uint32_t *fault = nullptr;
     int st = device_ctx(stream, ctx, &fault);
     if (st != RABIT_OK) return st;
-    return finish_launch(rabit::launch_svid_init(ctx, W, ldw, N, K, P, T, power_iters, s_in, s_out, alpha_in,
-                                                 alpha_out, a, b, packed, workspace, fault, wait_timeout_ns()));
+    return finish_launch(rabit::launch_svid_init(ctx, W, ldw, N, K, P, T, power_iters, power_tol, s_in, s_out, alpha_in,
+                                                 alpha_out, a, b, packed, workspace, fault, wait_timeout_ns(),
+                                                 env_flag("RABIT_TEST_SVID_WITHHOLD_ARRIVAL") ? 1 : 0));
 }
 
 int rabit_read_fault(void *stream, uint32_t *flags, int clear) {

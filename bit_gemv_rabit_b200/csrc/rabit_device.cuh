@@ -24,6 +24,7 @@ enum : uint32_t {
     FAULT_GEMV_WAIT_COPY = 1u << 5,
     FAULT_GEMV_WAIT_MMA = 1u << 6,
     FAULT_SCALE_GRADS_WAIT = 1u << 7,
+    FAULT_SVID_BARRIER = 1u << 8,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

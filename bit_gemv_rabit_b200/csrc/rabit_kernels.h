@@ -83,9 +83,9 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
 // Iterative Residual SVID initialisation (svid.cu).
 size_t svid_workspace_bytes(int N, int K, int P);
 cudaError_t launch_svid_init(const LaunchCtx &ctx, const float *W, int ldw, int N, int K, int P, int T,
-                             int power_iters, const float *s_in, const float *s_out, float alpha_in,
-                             float alpha_out, float *a, float *b, uint32_t *packed, void *workspace,
-                             uint32_t *fault_word, uint64_t timeout_ns);
+                             int power_iters, float power_tol, const float *s_in, const float *s_out,
+                             float alpha_in, float alpha_out, float *a, float *b, uint32_t *packed,
+                             void *workspace, uint32_t *fault_word, uint64_t timeout_ns, int debug = 0);
 
 size_t gemm_workspace_bytes(int N, int K, int P, int M);
 // Up to 4 layers with the same token count in one launch (gemm.cu); x of each layer is bf16.

@@ -39,8 +39,8 @@ SIGNATURES = [
     ("rabit_scale_grads_workspace_bytes", _sz, [_i, _i, _i]),
     ("rabit_scale_grads", _i, [_p, _i, _p, _p, _p, _i, _i, _i, _p, _p, _p, _sz, _p]),
     ("rabit_svid_init_workspace_bytes", _sz, [_i, _i, _i]),
-    ("rabit_svid_init", _i, [_p, _i, _i, _i, _i, _i, _i, _p, _p, ctypes.c_float, ctypes.c_float,
-                             _p, _p, _p, _p, _sz, _p]),
+    ("rabit_svid_init", _i, [_p, _i, _i, _i, _i, _i, _i, ctypes.c_float, _p, _p, ctypes.c_float,
+                             ctypes.c_float, _p, _p, _p, _p, _sz, _p]),
     ("rabit_read_fault", _i, [_p, ctypes.POINTER(ctypes.c_uint32), _i]),
     ("rabit_last_cuda_error", _i, []),
     ("rabit_status_string", ctypes.c_char_p, [_i]),
@@ -282,12 +282,14 @@ def alloc_svid_init_workspace(N: int, K: int, P: int = 2, device=None) -> torch.
 def rabit_svid_init(W: torch.Tensor, s_in: torch.Tensor, s_out: torch.Tensor, alpha_in: float,
                     alpha_out: float, a: torch.Tensor, b: torch.Tensor, packed: torch.Tensor,
                     workspace: torch.Tensor, P: int = 2, T: int = 20, power_iters: int = 40,
-                    stream=None):
+                    power_tol: float = 0.0, stream=None):
     """W [N][K] fp32 (pitch W.stride(0)); s_in [K], s_out [N] fp32; a [P][N], b [P][K] fp32 and
-    packed (the final signs) out.  Iterative Residual SVID initialisation."""
+    packed (the final signs) out.  Iterative Residual SVID initialisation; each update takes
+    at most `power_iters` power steps, fewer once a step moves the unit vectors u and v by at
+    most `power_tol` (Euclidean norm)."""
     N, K = W.shape
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(load().rabit_svid_init(_dptr(W), N, K, W.stride(0), P, T, power_iters, _dptr(s_in),
+    _check(load().rabit_svid_init(_dptr(W), N, K, W.stride(0), P, T, power_iters, float(power_tol), _dptr(s_in),
                                   _dptr(s_out), float(alpha_in), float(alpha_out), _dptr(a), _dptr(b),
                                   _dptr(packed), _dptr(workspace), ws_bytes, _stream(stream)),
            "rabit_svid_init")

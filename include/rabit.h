@@ -301,8 +301,13 @@ RABIT_API int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed,
  *     a[i] = g_i' / s_out^alpha_out,   b[i] = h_i' / s_in^alpha_in
  * SVID is read as the sign-value-independent decomposition (sign plus the best rank-1
  * approximation of |R|), which the pages cite but do not define.  The leading singular
- * pair comes from `power_iters` power steps per update (fp32, deterministic order),
- * warm-started from the path's pair of the previous iteration (uniform vectors at t = 1).
+ * pair comes from power steps per update (fp32 sums, double norms, every sum in a fixed
+ * order, so the result is deterministic), warm-started from the path's pair of the previous
+ * iteration (uniform vectors at t = 1): at most `power_iters` of them, fewer when
+ * power_tol > 0 and a step moved both unit vectors u and v by at most power_tol (Euclidean
+ * norm): the step after it is the last (power_tol = 0: exactly power_iters steps).  Every
+ * step of an update runs inside one cooperative launch (one CTA per SM, two grid barriers
+ * per step, each wait bounded: an expired wait sets the fault word, see rabit_read_fault).
  * The pages use T = 20.
  *   W        [N][ldw] fp32, ldw >= K (input)
  *   s_in [K], s_out [N]  positive fp32 calibration statistics (inputs; the reconstruction
@@ -314,15 +319,16 @@ RABIT_API int rabit_scale_grads(const float *G, int ldg, const uint32_t *packed,
  *   workspace  at least rabit_svid_init_workspace_bytes(N, K, P) bytes (about 4*N*K),
  *              256-byte aligned, caller-owned, no initialisation needed.  Calls sharing it
  *              must not overlap.
- * Enqueues about T * P * (1 + 3 * power_iters) kernels on `stream` and returns.
- * Errors: INVALID_ARG (null, non-finite alpha), SHAPE (N, K < 1, ldw < K, T or power_iters
- *         outside 1..RABIT_SVID_MAX_ITERS), UNSUPPORTED (P not 2 or 3), ALIGNMENT (packed,
- *         workspace), WORKSPACE, ARCH, CUDA.
+ * Enqueues 2 + 2 * T * P kernels on `stream` (a residual pass and a power launch per update)
+ * and returns.
+ * Errors: INVALID_ARG (null, non-finite alpha, power_tol negative or not finite), SHAPE (N, K < 1,
+ *         ldw < K, T or power_iters outside 1..RABIT_SVID_MAX_ITERS), UNSUPPORTED (P not 2 or 3),
+ *         ALIGNMENT (packed, workspace), WORKSPACE, ARCH, CUDA.
  */
 #define RABIT_SVID_MAX_ITERS 1000
 RABIT_API size_t rabit_svid_init_workspace_bytes(int N, int K, int P);
 RABIT_API int rabit_svid_init(const float *W, int N, int K, int ldw, int P, int T, int power_iters,
-                              const float *s_in, const float *s_out, float alpha_in, float alpha_out,
+                              float power_tol, const float *s_in, const float *s_out, float alpha_in, float alpha_out,
                               float *a, float *b, uint32_t *packed, void *workspace,
                               size_t workspace_bytes, void *stream);
 

@@ -154,12 +154,15 @@ def test_svid_init_validation(lib):
     assert need >= 8 * 16 * 4                         # the residual alone
     assert lib.rabit_svid_init_workspace_bytes(8, 16, 4) == 0
     args = lambda **kw: [P(kw.get("W", FAKE)), kw.get("N", 8), kw.get("K", 16), kw.get("ldw", 16), kw.get("P", 2),
-                         kw.get("T", 20), kw.get("iters", 40), P(FAKE), P(FAKE), kw.get("ai", 0.8),
+                         kw.get("T", 20), kw.get("iters", 40), kw.get("tol", 0.0), P(FAKE), P(FAKE), kw.get("ai", 0.8),
                          kw.get("ao", 0.65), P(FAKE), P(FAKE), P(kw.get("packed", FAKE)),
                          P(kw.get("ws", FAKE)), kw.get("wsb", need), None]
     assert f(*args(W=0)) == INVALID
     assert f(*args(ai=float("nan"))) == INVALID
     assert f(*args(ao=float("inf"))) == INVALID
+    assert f(*args(tol=-1e-6)) == INVALID
+    assert f(*args(tol=float("nan"))) == INVALID
+    assert f(*args(tol=float("inf"))) == INVALID
     assert f(*args(N=0)) == SHAPE
     assert f(*args(ldw=15)) == SHAPE
     assert f(*args(T=0)) == SHAPE
@@ -179,7 +182,7 @@ def test_valid_arguments_without_gpu_fail_cleanly(lib):
     flags = ctypes.c_uint32(0)
     assert lib.rabit_read_fault(None, ctypes.byref(flags), 0) in (CUDA, ARCH)
     need = lib.rabit_svid_init_workspace_bytes(8, 16, 2)
-    st = lib.rabit_svid_init(P(FAKE), 8, 16, 16, 2, 20, 40, P(FAKE), P(FAKE), 0.8, 0.65, P(FAKE), P(FAKE),
+    st = lib.rabit_svid_init(P(FAKE), 8, 16, 16, 2, 20, 40, 0.0, P(FAKE), P(FAKE), 0.8, 0.65, P(FAKE), P(FAKE),
                              P(FAKE), P(FAKE), need, None)
     assert st in (CUDA, ARCH)
 

@@ -3,7 +3,9 @@
 Host-side test switches withhold one event a kernel waits for:
   - RABIT_TEST_SKIP_ONE_ARRIVE: the GEMM's expansion warps skip their first arrival;
   - RABIT_TEST_GEMV_WITHHOLD_COPY: the decode kernel's producer never issues its first copy;
-  - RABIT_TEST_SCALE_GRADS_WITHHOLD_COPY: the scale-gradient producer never issues its first box.
+  - RABIT_TEST_SCALE_GRADS_WITHHOLD_COPY: the scale-gradient producer never issues its first box;
+  - RABIT_TEST_SVID_WITHHOLD_ARRIVAL: CTA 0 of each SVID power launch skips its first
+    grid-barrier arrival.
 The bounded wait that depends on it expires (after RABIT_WAIT_TIMEOUT_MS); the kernel drains
 its in-flight copies, frees tensor memory and returns; the host reads RABIT_ERR_TIMEOUT with
 that wait's fault bit, and the next call on the same context is correct.  No GPU fault is
@@ -29,6 +31,7 @@ FAULT_GEMM_WAITS = (1 << 0) | (1 << 1) | (1 << 2) | (1 << 3)
 # expansion-group barrier; the MMA issuer starts waiting first, so its bit is usually the one
 FAULT_GEMV_WAITS = (1 << 5) | (1 << 6)
 FAULT_SCALE_GRADS_WAIT = 1 << 7
+FAULT_SVID_BARRIER = 1 << 8
 RABIT_ERR_TIMEOUT = -8
 
 
@@ -134,3 +137,32 @@ def test_scale_grads_copy_wait_expiry_is_reported_and_the_context_survives(monke
     for got, ref in ((ga, ref_a), (gb, ref_b)):
         err = float(np.max(np.abs(got.cpu().numpy() - ref)) / np.max(np.abs(ref)))
         assert err <= 1e-5
+
+
+def test_svid_barrier_expiry_is_reported_and_the_context_survives(monkeypatch):
+    from oracle import svid as osvid
+    N, K, P, T = 192, 320, 2, 2
+    W = inputs.weight(4500, N, K, outlier_frac=0.01)
+    s_in, s_out = inputs.calibration_stats(4500, N, K)
+    dev = lambda v: torch.from_numpy(np.ascontiguousarray(v)).cuda()
+    Wt, si, so = dev(W), dev(s_in), dev(s_out)
+    a, b = torch.empty((P, N), device="cuda"), torch.empty((P, K), device="cuda")
+    packed = rabit.alloc_packed(N, K, P=P)
+    ws = rabit.alloc_svid_init_workspace(N, K, P)
+    monkeypatch.setenv("RABIT_TEST_SVID_WITHHOLD_ARRIVAL", "1")
+    monkeypatch.setenv("RABIT_WAIT_TIMEOUT_MS", "50")
+    rabit.rabit_svid_init(Wt, si, so, 0.8, 0.65, a, b, packed, ws, P=P, T=T, power_iters=20)
+    st, flags = _read_fault()
+    assert st == RABIT_ERR_TIMEOUT
+    assert flags & FAULT_SVID_BARRIER
+    monkeypatch.delenv("RABIT_TEST_SVID_WITHHOLD_ARRIVAL")
+    monkeypatch.delenv("RABIT_WAIT_TIMEOUT_MS")
+    rabit.rabit_svid_init(Wt, si, so, 0.8, 0.65, a, b, packed, ws, P=P, T=T, power_iters=100)
+    torch.cuda.synchronize()
+    assert rabit.rabit_read_fault(clear=True) == 0
+    So, ao, bo = osvid.svid_init(W, s_in, s_out, 0.8, 0.65, P=P, T=T)
+    S = oracle.unpack(packed.cpu().numpy(), N, K, P=P)
+    rec, ref = osvid.reconstruct(S, a.cpu().numpy(), b.cpu().numpy()), osvid.reconstruct(So, ao, bo)
+    agree = np.all(S == So, axis=0)          # (a residual within rounding of 0 may flip)
+    assert np.mean(~agree) <= 1e-4
+    assert float(np.linalg.norm((rec - ref)[agree]) / np.linalg.norm(ref)) <= 1e-4

@@ -7,7 +7,9 @@ sigma_2/sigma_1, about 0.5 on these inputs) the two agree to fp32 rounding.  Tol
 derived from the arithmetic: fp32 sums over K terms (about sqrt(K) * 2^-24 relative) carried
 through T iterations stay below 1e-5 in a float32 emulation of the same steps on these
 inputs, so the scales and the reconstruction must agree within 1e-4 (Frobenius, relative),
-and at most 1e-4 of the signs may differ (residual elements within rounding of 0).
+and at most 1e-4 of the signs may differ (residual elements within rounding of 0).  One
+such flip moves its element by 2 |a b|, which on a large matrix alone exceeds 1e-4 of the
+norm, so the reconstruction is compared where every path's sign agrees.
 """
 import numpy as np
 import pytest
@@ -40,7 +42,14 @@ def fro(x, ref):
     return float(np.linalg.norm(np.asarray(x, np.float64) - ref) / np.linalg.norm(ref))
 
 
-def gpu_init(W, s_in, s_out, P, T, power_iters=100, ldw=None):
+def recon_err(S, a, b, So, ao, bo):
+    """Relative Frobenius error of the reconstruction where all paths' signs agree."""
+    rec, ref = osvid.reconstruct(S, a, b), osvid.reconstruct(So, ao, bo)
+    agree = np.all(S == So, axis=0)
+    return float(np.linalg.norm((rec - ref)[agree]) / np.linalg.norm(ref))
+
+
+def gpu_init(W, s_in, s_out, P, T, power_iters=100, ldw=None, power_tol=0.0):
     N, K = W.shape
     if ldw is None:
         Wt = torch.from_numpy(W).cuda()
@@ -54,13 +63,16 @@ def gpu_init(W, s_in, s_out, P, T, power_iters=100, ldw=None):
     packed.view(torch.int32).fill_(-0x5A5A5A5B)   # 0xA5A5A5A5: every word must be written
     ws = rabit.alloc_svid_init_workspace(N, K, P)
     rabit.rabit_svid_init(Wt, torch.from_numpy(s_in).cuda(), torch.from_numpy(s_out).cuda(), ALPHA_IN,
-                          ALPHA_OUT, a, b, packed, ws, P=P, T=T, power_iters=power_iters)
+                          ALPHA_OUT, a, b, packed, ws, P=P, T=T, power_iters=power_iters, power_tol=power_tol)
     torch.cuda.synchronize()
     return a.cpu().numpy(), b.cpu().numpy(), packed.cpu().numpy()
 
 
+# (1000, 9001): three column sweeps of the power launch, the last ragged; (64, 96): fewer rows
+# than CTAs, so some CTAs own no row
 @pytest.mark.parametrize("N,K,P,T", [(64, 96, 2, 3), (100, 203, 3, 2), (256, 512, 2, 20),
-                                     (256, 512, 3, 20), (1024, 4096, 2, 3)])
+                                     (256, 512, 3, 20), (1024, 4096, 2, 3), (1000, 9001, 2, 2),
+                                     (3000, 257, 3, 2)])
 def test_svid_init_matches_oracle(N, K, P, T):
     W = inputs.weight(21 + N, N, K, outlier_frac=0.01)
     s_in, s_out = inputs.calibration_stats(21 + N, N, K)
@@ -72,7 +84,7 @@ def test_svid_init_matches_oracle(N, K, P, T):
     column_bits = oracle.pack(-np.ones_like(So))
     assert not np.any(packed.view(np.uint32) & ~column_bits)
     assert fro(a, ao) <= TOL and fro(b, bo) <= TOL
-    assert fro(osvid.reconstruct(S, a, b), osvid.reconstruct(So, ao, bo)) <= TOL
+    assert recon_err(S, a, b, So, ao, bo) <= TOL
 
 
 def test_svid_init_recovers_preconditioned_signed_rank1():
@@ -118,3 +130,18 @@ def test_svid_init_degenerate_cases():
     for i, sig in enumerate([3.0, 2.0, 1.0]):
         np.testing.assert_allclose(a[i], np.sqrt(sig) * np.eye(3)[i], atol=1e-5)
         np.testing.assert_allclose(b[i], np.sqrt(sig) * np.eye(3)[i], atol=1e-5)
+
+
+def test_svid_init_settled_stop_matches_oracle():
+    """With a relative tolerance on sigma the power steps stop early; the result still meets
+    the oracle's bar, and is deterministic."""
+    N, K, P, T = 512, 768, 2, 6
+    W = inputs.weight(77, N, K, outlier_frac=0.01)
+    s_in, s_out = inputs.calibration_stats(77, N, K)
+    So, ao, bo = osvid.svid_init(W, s_in, s_out, ALPHA_IN, ALPHA_OUT, P=P, T=T)
+    a, b, packed = gpu_init(W, s_in, s_out, P, T, power_iters=400, power_tol=1e-6)
+    a2, b2, p2 = gpu_init(W, s_in, s_out, P, T, power_iters=400, power_tol=1e-6)
+    assert np.array_equal(a, a2) and np.array_equal(b, b2) and np.array_equal(packed, p2)
+    S = oracle.unpack(packed, N, K, P=P)
+    assert np.mean(S != So) <= SIGN_TOL
+    assert recon_err(S, a, b, So, ao, bo) <= TOL
