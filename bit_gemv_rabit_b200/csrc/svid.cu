@@ -14,10 +14,10 @@
 // sign-value-independent decomposition this is.
 //
 // Design (HBM-bound passes, CUDA cores):
-//  * Residual pass, once per (t, i): a warp per 32-column group reads the group's W values
-//    (128 contiguous bytes), the other paths' packed words (one broadcast load each) and
-//    scales, writes R (fp32, rows 16-byte aligned) and a ballot of the signs straight into
-//    path i of the packed output -- the same layout the decode and prefill kernels read.
+//  * Residual pass, once per (t, i): a warp per 128 columns of a row (two such pieces in
+//    flight) reads W, the other paths' packed words (broadcast loads) and the scales, writes
+//    R (fp32, rows 16-byte aligned) and the signs straight into path i of the packed output
+//    -- the same layout the decode and prefill kernels read.
 //  * Power iteration for (sigma, u, v), warm-started from the path's vectors of the previous
 //    iteration, in ONE cooperative launch per (t, i) that runs every power step.  A step is
 //    one pass over R that yields both u' = |R| v and v' = |R|^T u (|R| from R itself): CTA c
@@ -119,39 +119,79 @@ svid_prep_kernel(const float *__restrict__ s_in, const float *__restrict__ s_out
 }
 
 // R_i = W' - sum_{p != i} g_p' (.) B_p (.) h_p', its signs into path i of the packed output;
-// also resets the power launch's grid barrier.
-template <int kP>
+// also resets the power launch's grid barrier.  A warp takes 128 columns of a row (four
+// consecutive columns a lane, a float4 of W when its rows are 16-byte aligned) and two such
+// pieces at a time, so enough of W is in flight to stream it; eight lanes make one 32-column
+// sign word.
+template <int kP, bool kVecW>
 __global__ void __launch_bounds__(kThreads)
 svid_residual_kernel(const float *__restrict__ W, int ldw, int N, int K, int Wr, int path,
                      uint32_t *__restrict__ packed, SvidWs w) {
     constexpr int G = kP == 2 ? 2 : 4;  // words per 32-column group in the packed layout
     pdl_enter();
     if (blockIdx.x == 0 && threadIdx.x < 2) w.sync[threadIdx.x] = 0u;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, sub = lane & 7, grp = lane >> 3;
+    const int nblk = Wr / 4;                 // 128-column blocks per row (Wr is a multiple of 4)
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    const int64_t groups = static_cast<int64_t>(N) * Wr;
+    const int64_t units = static_cast<int64_t>(N) * nblk;
     const int64_t ldr = residual_pitch(K);
-    for (int64_t gi = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; gi < groups;
-         gi += nwarps) {
-        const int n = static_cast<int>(gi / Wr);
-        const int j = static_cast<int>(gi - static_cast<int64_t>(n) * Wr) * 32 + lane;
-        const bool ok = j < K;
-        float r = 0.0f;
-        if (ok) {
-            r = w.so[n] * __ldg(W + static_cast<int64_t>(n) * ldw + j) * w.si[j];
+    for (int64_t u0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u0 < units;
+         u0 += 2 * nwarps) {
+        float x[2][4];
 #pragma unroll
-            for (int p = 0; p < kP; ++p) {
-                if (p == path) continue;
-                const bool neg = (packed[gi * G + p] >> lane) & 1u;
-                const float m = w.gp[p * static_cast<int64_t>(N) + n] * w.hp[p * static_cast<int64_t>(K) + j];
-                r = neg ? r + m : r - m;
+        for (int h = 0; h < 2; ++h) {           // both pieces' loads go out first
+            const int64_t u = u0 + h * nwarps;
+            const int n = static_cast<int>(u / nblk);
+            const int j = static_cast<int>(u - static_cast<int64_t>(n) * nblk) * 128 + 4 * lane;
+            const float *src = W + static_cast<int64_t>(n) * ldw + j;
+            if (u < units && kVecW && j + 3 < K) {
+                const float4 v = __ldcs(reinterpret_cast<const float4 *>(src));
+                x[h][0] = v.x; x[h][1] = v.y; x[h][2] = v.z; x[h][3] = v.w;
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) x[h][q] = (u < units && j + q < K) ? __ldcs(src + q) : 0.0f;
             }
-            w.R[static_cast<int64_t>(n) * ldr + j] = r;
         }
-        const uint32_t bits = __ballot_sync(0xffffffffu, ok && r < 0.0f);   // sign(v) = -1 iff v < 0
-        if (lane == 0) {
-            packed[gi * G + path] = bits;
-            if (kP == 3 && path == 0) packed[gi * G + 3] = 0u;                 // padding word
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t u = u0 + h * nwarps;
+            if (u >= units) break;               // (warp-uniform)
+            const int n = static_cast<int>(u / nblk);
+            const int blk = static_cast<int>(u - static_cast<int64_t>(n) * nblk);
+            const int j = blk * 128 + 4 * lane;
+            const int64_t word = (static_cast<int64_t>(n) * Wr + blk * 4 + grp) * G;   // this lane's group
+            const float so = w.so[n];
+            uint32_t other[kP];
+#pragma unroll
+            for (int p = 0; p < kP; ++p) other[p] = p == path ? 0u : packed[word + p];
+            float r[4];
+            uint32_t nib = 0u;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                r[q] = 0.0f;
+                if (j + q < K) {
+                    float v = so * x[h][q] * w.si[j + q];
+#pragma unroll
+                    for (int p = 0; p < kP; ++p) {
+                        if (p == path) continue;
+                        const bool neg = (other[p] >> (4 * sub + q)) & 1u;
+                        const float m = w.gp[p * static_cast<int64_t>(N) + n] * w.hp[p * static_cast<int64_t>(K) + j + q];
+                        v = neg ? v + m : v - m;
+                    }
+                    r[q] = v;
+                    nib |= (v < 0.0f ? 1u : 0u) << q;    // sign(v) = -1 iff v < 0
+                }
+            }
+            if (j < K)                            // (the row pitch covers the whole float4)
+                *reinterpret_cast<float4 *>(w.R + static_cast<int64_t>(n) * ldr + j) = make_float4(r[0], r[1], r[2], r[3]);
+            uint32_t bits = nib << (4 * sub);     // the eight lanes of a group make its word
+            bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
+            bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
+            bits |= __shfl_xor_sync(0xffffffffu, bits, 4);
+            if (sub == 0) {
+                packed[word + path] = bits;
+                if (kP == 3 && path == 0) packed[word + 3] = 0u;                 // padding word
+            }
         }
     }
 }
@@ -162,13 +202,6 @@ __device__ __forceinline__ T warp_sum(T v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
-}
-
-// sum_i x[i]^2 over [0, n) in a fixed order (lane-strided, then the tree), by one warp.
-__device__ __forceinline__ double warp_sumsq(const float *x, int n, int lane) {
-    double s = 0.0;
-    for (int i = lane; i < n; i += 32) s += static_cast<double>(x[i]) * x[i];
-    return warp_sum(s);
 }
 
 constexpr int kPerLane = (kMaxPowGrid + 31) / 32;      // per-CTA values a lane adds up
@@ -218,8 +251,10 @@ __device__ bool grid_sync(const PowerArgs &p, unsigned target, int *s_ok) {
     __syncthreads();
     if (threadIdx.x == 0) {
         bool ok = true;
-        __threadfence();                       // this CTA's writes before its arrival
-        if (!(p.debug == 1 && blockIdx.x == 0 && target == gridDim.x)) atomicAdd(&p.w.sync[0], 1u);
+        // The CTA's writes (ordered before this thread's by the CTA barrier) are released with
+        // the arrival and acquired by every CTA that sees the count complete.
+        if (!(p.debug == 1 && blockIdx.x == 0 && target == gridDim.x))
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.w.sync[0]) : "memory");
         if (ld_acquire_gpu(&p.w.sync[0]) < target) {
             const uint64_t t0 = global_timer_ns();
             while (ld_acquire_gpu(&p.w.sync[0]) < target) {
@@ -233,7 +268,6 @@ __device__ bool grid_sync(const PowerArgs &p, unsigned target, int *s_ok) {
                 __nanosleep(32);
             }
         }
-        __threadfence();
         *s_ok = ok ? 1 : 0;
     }
     __syncthreads();
@@ -256,10 +290,12 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
     const SvidWs &w = p.w;
     float *U = w.U + p.path * static_cast<int64_t>(N), *V = w.V + p.path * static_cast<int64_t>(K);
     float *part = w.part + static_cast<int64_t>(c) * p.ldr;
+    const int64_t moved_off = 2 * kMaxPowGrid;     // slots [2], [3] of a parity: the moves
     bool v_from_acc = false;                   // current v: V, or v' / ||v'|| of the last step
     float ib_prev = 0.0f;
     unsigned target = 0;
     for (int s = 0; s < p.steps; ++s) {
+        double usq = 0.0;                      // this thread's part of |u'|^2 (own rows)
         // ---- pass over the CTA's rows: u'_n = sum_j |R_nj| v_j, column partials sum_n |R_nj| u_n
         for (int cb = 0; cb < K; cb += kPowChunk) {
             float4 vv[kPowVec], cp[kPowVec];
@@ -326,7 +362,9 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
                         float t = 0.0f;
 #pragma unroll
                         for (int q = 0; q < kPowWarps; ++q) t += red[q][i];
-                        w.uacc[nb + i] = cb == 0 ? t : w.uacc[nb + i] + t;   // same thread every sweep
+                        t = cb == 0 ? t : w.uacc[nb + i] + t;   // same thread every sweep
+                        w.uacc[nb + i] = t;
+                        if (cb + kPowChunk >= K) usq += static_cast<double>(t) * t;
                     }
                     __syncthreads();
                 }
@@ -337,17 +375,21 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
                 if (j < K) *reinterpret_cast<float4 *>(part + j) = cp[m];   // (part pitch = ldr)
             }
         }
-        double *nsq = w.nsq + static_cast<int64_t>(s & 1) * 4 * kMaxPowGrid;   // this step's sums
-        const double *moved = w.nsq + static_cast<int64_t>((s + 1) & 1) * 4 * kMaxPowGrid + 2 * kMaxPowGrid;
+        // this step's per-CTA sums: [0] |u'|^2, [1] |v'|^2, [2] [3] the moves of the step before
+        double *nsq = w.nsq + static_cast<int64_t>(s & 1) * 4 * kMaxPowGrid;
+        usq = warp_sum(usq);
+        if (lane == 0) red2[warp][0] = usq;
         __syncthreads();
-        if (warp == 0) {
-            const double t = warp_sumsq(w.uacc + r0, r1 - r0, lane);
-            if (lane == 0) nsq[c] = t;
+        if (tid == 0) {
+            double t = 0.0;
+            for (int q = 0; q < kPowWarps; ++q) t += red2[q][0];
+            nsq[c] = t;
         }
         target += static_cast<unsigned>(G);
         if (!grid_sync(p, target, &s_ok)) return;
         // ---- v'_j for this CTA's columns: the G partials added in CTA order (lane q mod 32
         // adds its CTAs in turn, then the tree), four columns per warp at a time
+        double vsq = 0.0;                      // lane 0: this warp's part of |v'|^2
         for (int jb = k0 + warp; jb < k1; jb += 4 * kPowWarps) {
             float v[4][kPerLane];
 #pragma unroll
@@ -364,23 +406,30 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
                 for (int i = 0; i < kPerLane; ++i) t += v[u][i];
                 t = warp_sum(t);
                 const int j = jb + u * kPowWarps;
-                if (lane == 0 && j < k1) w.vacc[j] = t;
+                if (lane == 0 && j < k1) {
+                    w.vacc[j] = t;
+                    vsq += static_cast<double>(t) * t;
+                }
             }
         }
+        if (lane == 0) red2[warp][1] = vsq;
         __syncthreads();
-        if (warp == 0) {
-            const double t = warp_sumsq(w.vacc + k0, k1 - k0, lane);
-            if (lane == 0) nsq[kMaxPowGrid + c] = t;
+        if (tid == 0) {
+            double t = 0.0;
+            for (int q = 0; q < kPowWarps; ++q) t += red2[q][1];
+            nsq[kMaxPowGrid + c] = t;
         }
         target += static_cast<unsigned>(G);
         if (!grid_sync(p, target, &s_ok)) return;
-        // ---- norms (every CTA the same), then normalise or finish
+        // ---- norms (every CTA the same), then normalise or finish.  This thread's first row
+        // and column are fetched while warp 0 adds the per-CTA sums.
+        const int nf = r0 + tid, jf = k0 + tid;
+        const float uf = nf < r1 ? w.uacc[nf] : 0.0f, uf_old = nf < r1 ? U[nf] : 0.0f;
+        const float vf = jf < k1 ? w.vacc[jf] : 0.0f, vf_old = jf < k1 ? V[jf] : 0.0f;
         if (warp == 0) {
-            double t[2], m[2] = {0.0, 0.0};
-            warp_totals<2>(nsq, G, lane, t);
-            // how far u and v moved in the previous step (written before this step's barriers)
-            if (s > 0) warp_totals<2>(moved, G, lane, m);
-            if (lane == 0) { nsh[0] = t[0]; nsh[1] = t[1]; nsh[2] = m[0]; nsh[3] = m[1]; }
+            double t[4];
+            warp_totals<4>(nsq, G, lane, t);   // the moves were written before this step's barriers
+            if (lane == 0) { nsh[0] = t[0]; nsh[1] = t[1]; nsh[2] = s > 0 ? t[2] : 0.0; nsh[3] = s > 0 ? t[3] : 0.0; }
         }
         __syncthreads();
         const double na = sqrt(nsh[0]), nb = sqrt(nsh[1]);
@@ -391,13 +440,13 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
         if (s == p.steps - 1 || settled) {
             const float rs = static_cast<float>(sqrt(na));    // sqrt(sigma)
             float *gp = w.gp + p.path * static_cast<int64_t>(N), *hp = w.hp + p.path * static_cast<int64_t>(K);
-            for (int n = r0 + tid; n < r1; n += kPowThreads) {
-                const float u = w.uacc[n] * ia;
+            for (int n = nf; n < r1; n += kPowThreads) {
+                const float u = (n == nf ? uf : w.uacc[n]) * ia;
                 gp[n] = rs * u;
                 if (na > 0.0) U[n] = u;
             }
-            for (int j = k0 + tid; j < k1; j += kPowThreads) {
-                const float v = w.vacc[j] * ib;
+            for (int j = jf; j < k1; j += kPowThreads) {
+                const float v = (j == jf ? vf : w.vacc[j]) * ib;
                 hp[j] = nb > 0.0 ? rs * v : 0.0f;
                 if (nb > 0.0) V[j] = v;
             }
@@ -405,18 +454,19 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
         }
         // A zero product keeps the old vector.  V is read by other CTAs only while the last
         // step's v' is zero, and then nobody writes it.  The squared moves of this CTA's
-        // rows of u and columns of v go to the next step's decision.
+        // rows of u and columns of v go to the next step's decision (slots [2], [3] of the
+        // next step's parity).
         double du = 0.0, dv = 0.0;
         if (na > 0.0)
-            for (int n = r0 + tid; n < r1; n += kPowThreads) {
-                const float u = w.uacc[n] * ia;
-                du += static_cast<double>(u - U[n]) * (u - U[n]);
+            for (int n = nf; n < r1; n += kPowThreads) {
+                const float u = (n == nf ? uf : w.uacc[n]) * ia, uo = n == nf ? uf_old : U[n];
+                du += static_cast<double>(u - uo) * (u - uo);
                 U[n] = u;
             }
         if (nb > 0.0)
-            for (int j = k0 + tid; j < k1; j += kPowThreads) {
-                const float v = w.vacc[j] * ib;
-                dv += static_cast<double>(v - V[j]) * (v - V[j]);
+            for (int j = jf; j < k1; j += kPowThreads) {
+                const float v = (j == jf ? vf : w.vacc[j]) * ib, vo = j == jf ? vf_old : V[j];
+                dv += static_cast<double>(v - vo) * (v - vo);
                 V[j] = v;
             }
         du = warp_sum(du);
@@ -426,8 +476,9 @@ svid_power_kernel(const __grid_constant__ PowerArgs p) {
         if (tid == 0) {
             double su = 0.0, sv = 0.0;
             for (int q = 0; q < kPowWarps; ++q) { su += red2[q][0]; sv += red2[q][1]; }
-            nsq[2 * kMaxPowGrid + c] = su;
-            nsq[3 * kMaxPowGrid + c] = sv;
+            double *next = w.nsq + static_cast<int64_t>((s + 1) & 1) * 4 * kMaxPowGrid;
+            next[moved_off + c] = su;
+            next[moved_off + kMaxPowGrid + c] = sv;
         }
         v_from_acc = nb > 0.0;
         if (v_from_acc) ib_prev = ib;
@@ -475,9 +526,10 @@ cudaError_t launch_svid_init(const LaunchCtx &ctx, const float *W, int ldw, int 
     const int Wr = static_cast<int>(padded_cols(K) / 32);
     const int64_t vec_len = std::max<int64_t>(N, K);
     const int vec_grid = static_cast<int>(std::min<int64_t>((vec_len + kThreads - 1) / kThreads, ctx.num_sms * 4));
-    const int64_t warps = static_cast<int64_t>(N) * Wr;
+    const int64_t warps = static_cast<int64_t>(N) * (Wr / 4);    // one per 128 columns of a row
     const int res_grid = static_cast<int>(std::min<int64_t>((warps * 32 + kThreads - 1) / kThreads,
                                                             static_cast<int64_t>(ctx.num_sms) * 16));
+    const bool vec_w = reinterpret_cast<uintptr_t>(W) % 16 == 0 && ldw % 4 == 0;
     // The power launch's CTAs wait on one another, so all must be resident: one per SM.
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, svid_power_kernel, kPowThreads, 0);
@@ -507,8 +559,10 @@ cudaError_t launch_svid_init(const LaunchCtx &ctx, const float *W, int ldw, int 
     e = launch(ctx, vec_grid, kThreads, svid_prep_kernel, s_in, s_out, alpha_in, alpha_out, N, K, P, w);
     for (int t = 0; t < T && e == cudaSuccess; ++t) {
         for (int i = 0; i < P && e == cudaSuccess; ++i) {
-            e = P == 2 ? launch(ctx, res_grid, kThreads, svid_residual_kernel<2>, W, ldw, N, K, Wr, i, packed, w)
-                       : launch(ctx, res_grid, kThreads, svid_residual_kernel<3>, W, ldw, N, K, Wr, i, packed, w);
+            void (*res)(const float *, int, int, int, int, int, uint32_t *, SvidWs) =
+                P == 2 ? (vec_w ? svid_residual_kernel<2, true> : svid_residual_kernel<2, false>)
+                       : (vec_w ? svid_residual_kernel<3, true> : svid_residual_kernel<3, false>);
+            e = launch(ctx, res_grid, kThreads, res, W, ldw, N, K, Wr, i, packed, w);
             if (e != cudaSuccess) break;
             pa.path = i;
             e = cudaLaunchKernelEx(&pcfg, svid_power_kernel, pa);
