@@ -957,18 +957,18 @@ gemv_tc_kernel(const __grid_constant__ GArgs p) {
                     for (int beta = 0; beta < kMaxBatch; ++beta)
                         if (beta < p.nb) slot[beta * tile_rows + hh * kRows + row] = ypart[hh][beta];
                 }
-            // Every thread's partial stores are fenced, then one counter increment (acquire and
-            // release at GPU scope) tells the last contributor that every partial is visible.
-            __threadfence();
+            // The group barrier orders every thread's partial stores before the counting
+            // thread's fence and increment (acquire and release at GPU scope), which tell the
+            // last contributor that every partial is visible.
             if (!group_sync(ctl, gphase, lane, p)) break;
             if (gt == 0) {
+                __threadfence();
                 int old;
                 asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(&p.tickets[gtile]) : "memory");
                 ctl->last = (old == lastc - first) ? 1 : 0;
             }
             if (!group_sync(ctl, gphase, lane, p)) break;
             if (ctl->last) {
-                __threadfence();
                 // The partials of contributors first..lastc, added in that (column) order.
                 // Loads go out eight at a time so their latencies overlap.  Every contributor
                 // but the first starts its range inside this tile, so this tile is its first
