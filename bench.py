@@ -60,7 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=400)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the GEMM / derive / CPU-baseline measurements")
-    ap.add_argument("--profile-kernel", choices=["derive", "gemv", "gemv_set", "gemm", "svid"], default=None,
+    ap.add_argument("--profile-kernel", choices=["derive", "gemv", "gemv_set", "gemm", "svid", "scale_grads"],
+                    default=None,
                     help="run a few launches of one kernel (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=3, metavar=("N", "K", "M"), default=(11008, 4096, 1),
                     help="with --profile-kernel: out features, in features, batch/tokens")
@@ -915,6 +916,12 @@ def profile_kernel(args):
     L = make_layer(rabit, spec, 0, "layer", N, K, device, M)
     W = torch.from_numpy(inputs.weight(inputs.seed_for(9, 0), N, K)).to(device)
     ws = rabit.alloc_gemm_workspace(N, K, 2, M, device=device) if args.profile_kernel == "gemm" else None
+    if args.profile_kernel == "scale_grads":
+        # G = dL/dW_hat, seeded Gaussian (fp32, N x K); --launches calls
+        G = torch.randn((N, K), generator=torch.Generator().manual_seed(inputs.seed_for(9, 1)),
+                        dtype=torch.float32).to(device)
+        ga, gb = torch.empty((2, N), device=device), torch.empty((2, K), device=device)
+        ws = rabit.alloc_scale_grads_workspace(N, K, 2, device=device)
     if args.profile_kernel == "svid":
         # one initialisation: T = --launches iterations, 5 power steps per update
         s_in, s_out = inputs.calibration_stats(inputs.seed_for(9, 0), N, K)
@@ -927,6 +934,8 @@ def profile_kernel(args):
             rabit.rabit_derive_pack(W, L["a"], L["b"], L["packed"])
         elif args.profile_kernel == "gemv":
             rabit.rabit_gemv(L["packed"], L["a"], L["b"], N, K, L["x"], L["y"], workspace=L["ws"])
+        elif args.profile_kernel == "scale_grads":
+            rabit.rabit_scale_grads(G, L["packed"], L["a"], L["b"], N, K, ga, gb, ws)
         else:
             rabit.rabit_gemm(L["packed"], L["a"], L["b"], N, K, L["x"], L["y"], ws)
     torch.cuda.synchronize()
