@@ -72,9 +72,12 @@ class RowShard:
             rabit.rabit_gemv(self.packed, self.a, self.b, self.rows, self.K, x, local[:, :self.rows], P=self.P)
         return local
 
-    def gemv(self, x: torch.Tensor, y: torch.Tensor, group=None) -> torch.Tensor:
+    def gemv(self, x: torch.Tensor, y: torch.Tensor, group=None, check_fault: bool = True) -> torch.Tensor:
         """y[:, n] for all n of the layer, from this rank's rows and one all-gather.
-        Every rank of the group must call it (ranks without rows still join the gather)."""
+        Every rank of the group must call it (ranks without rows still join the gather).
+        With check_fault, a rank whose kernel had a bounded wait expire raises RabitError
+        after the gather (so every rank still takes the same collective steps); this
+        synchronises the rank's stream once per call."""
         import torch.distributed as dist
         batch = x.shape[0]
         local = self.local(x)
@@ -85,4 +88,8 @@ class RowShard:
         for r in range(self.world):
             b0, b1 = row_block(self.N, self.world, r)
             y[:, b0:b1] = gathered[r, :, :b1 - b0]
+        if check_fault and self.rows:
+            fault = rabit.rabit_read_fault(clear=True)
+            if fault:
+                raise rabit.RabitError(-8, f"RowShard.gemv (rank {self.rank}, fault word {fault:#x})")
         return y

@@ -60,6 +60,7 @@ def _worker(rank, world, port, N, K, B, use_derive, out):
         return packed
 
     rabit.rabit_gemv = fake_gemv
+    rabit.rabit_read_fault = lambda clear=True, stream=None: 0   # no device here
     rabit.rabit_derive_pack = fake_derive
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     try:
