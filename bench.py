@@ -770,21 +770,35 @@ def run_ours(args, rank, world, local, dist):
     # every bounded device wait of the timed region must have completed
     fault = rabit.rabit_read_fault(clear=True)
 
-    # ---- end to end through the public API: pinned host x in, y back to the host, per step
+    # ---- end to end through the public API: pinned host x in, y back to the host, per step.
+    # Each copy of the set keeps its seven x and seven y as views of one device buffer each,
+    # so a step is one host-to-device copy, one prepared grouped call (rabit.GemvGroup, the
+    # binding's marshalled rabit_gemv_grouped) and one device-to-host copy.
     e2e_steps = min(args.e2e_steps, args.steps)
-    x_pinned = [torch.from_numpy(L["x_host"].view(np.int16)).view(torch.bfloat16).pin_memory() for L in base]
-    y_pinned = [torch.empty_like(L["y"], device="cpu").pin_memory() for L in base]
-    h2d = sum(x.numel() * x.element_size() for x in x_pinned)
-    d2h = sum(y.numel() * y.element_size() for y in y_pinned)
+    x_pinned = torch.from_numpy(np.concatenate([L["x_host"].view(np.int16).reshape(-1) for L in base])
+                                ).view(torch.bfloat16).pin_memory()
+    n_out = sum(L["N"] for L in base)
+    y_pinned = torch.empty(n_out, dtype=torch.float32).pin_memory()
+    h2d = x_pinned.numel() * x_pinned.element_size()
+    d2h = y_pinned.numel() * y_pinned.element_size()
+    e2e_sets = []
+    for layers in sets:
+        xd = torch.empty(x_pinned.numel(), dtype=torch.bfloat16, device=device)
+        yd = torch.empty(n_out, dtype=torch.float32, device=device)
+        tup, xo, yo = [], 0, 0
+        for L in layers:
+            tup.append((L["packed"], L["a"], L["b"], L["N"], L["K"], xd[xo:xo + L["K"]].view(1, L["K"]),
+                        yd[yo:yo + L["N"]].view(1, L["N"])))
+            xo += L["K"]
+            yo += L["N"]
+        e2e_sets.append((xd, yd, rabit.GemvGroup(tup, workspace=ws)))
     stream = torch.cuda.current_stream()
 
     def e2e_step(s):
-        layers = sets[s % COPIES]
-        for L, xp in zip(layers, x_pinned):
-            L["x"].copy_(xp, non_blocking=True)
-        rabit.rabit_gemv_grouped(layer_tuples(layers), workspace=ws)
-        for L, yp in zip(layers, y_pinned):
-            yp.copy_(L["y"], non_blocking=True)
+        xd, yd, group = e2e_sets[s % COPIES]
+        xd.copy_(x_pinned, non_blocking=True)
+        group.run(stream)
+        y_pinned.copy_(yd, non_blocking=True)
         stream.synchronize()
 
     for s in range(5):
@@ -827,8 +841,9 @@ def run_ours(args, rank, world, local, dist):
         "fault_word": fault,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "api": "bit_gemv_rabit_b200.rabit.rabit_gemv_grouped over the set, pinned host copies, "
-                       "stream sync per step"},
+                "api": "bit_gemv_rabit_b200.rabit.GemvGroup.run (a prepared rabit_gemv_grouped) over the "
+                       "set; one pinned host-to-device copy of the seven x and one device-to-host copy "
+                       "of the seven y per step, then a stream sync"},
     }
     if clocks is not None:
         line["clocks"] = clocks.summary()

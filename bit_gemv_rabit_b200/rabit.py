@@ -183,6 +183,29 @@ def rabit_gemv_grouped(layers, P: int = 2, workspace: torch.Tensor | None = None
     return [layer[6] for layer in layers]
 
 
+class GemvGroup:
+    """A prepared rabit_gemv_grouped call over fixed tensors: the layer array, the scalar
+    arguments and the workspace are marshalled once, and run() only enqueues.  The layers'
+    tensors (kept referenced here) must stay the same objects; their contents may change
+    between runs (new x every step, say)."""
+
+    def __init__(self, layers, P: int = 2, workspace: torch.Tensor | None = None):
+        self.layers = list(layers)
+        self._arr = _layer_array(self.layers)
+        self._ptr = ctypes.cast(self._arr, ctypes.c_void_p)
+        x0 = self.layers[0][5]
+        self._scalars = (len(self.layers), P, _dtype_code(x0), x0.shape[0])
+        if workspace is None:
+            workspace = alloc_gemv_grouped_workspace(self.layers, P, device=x0.device)
+        self.workspace = workspace
+        self._ws = (_dptr(workspace), workspace.numel() * workspace.element_size())
+        self._fn = load().rabit_gemv_grouped
+
+    def run(self, stream=None):
+        _check(self._fn(self._ptr, *self._scalars, *self._ws, _stream(stream)), "rabit_gemv_grouped")
+        return [layer[6] for layer in self.layers]
+
+
 def rabit_gemm(packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, N: int, K: int,
                x: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor, P: int = 2,
                stream=None) -> torch.Tensor:

@@ -104,3 +104,37 @@ def test_grouped_llama2_7b_decode_set_one_launch():
         torch.cuda.synchronize()
         for L in layers:
             assert normwise(L["y"].cpu().numpy().astype(np.float64), L["ref"]) <= 2e-3
+
+
+def test_prepared_group_matches_the_plain_call_as_x_changes():
+    """GemvGroup marshals the call once; each run reads the tensors' current contents, so new
+    x (written in place, as an end-to-end step does) gives the plain call's y bit for bit,
+    and y meets the oracle's bar.  x and y are views of one flat buffer each."""
+    shapes = [(4096, 4096), (1024, 4096), (512, 11008)]
+    layers = [_layer(7300 + i, N, K, 1, torch.bfloat16) for i, (N, K) in enumerate(shapes)]
+    xflat = torch.empty(sum(K for _, K in shapes), dtype=torch.bfloat16, device="cuda")
+    yflat = torch.empty(sum(N for N, _ in shapes), dtype=torch.float32, device="cuda")
+    tup, xo, yo = [], 0, 0
+    for L in layers:
+        tup.append((L["packed"], L["a"], L["b"], L["N"], L["K"], xflat[xo:xo + L["K"]].view(1, L["K"]),
+                    yflat[yo:yo + L["N"]].view(1, L["N"])))
+        xo += L["K"]
+        yo += L["N"]
+    group = rabit.GemvGroup(tup)
+    for step in range(2):
+        xs = [inputs.activations(7400 + 10 * step + i, 1, K) for i, (_, K) in enumerate(shapes)]
+        xflat.copy_(torch.from_numpy(np.concatenate([x.view(np.int16).reshape(-1) for x in xs]))
+                    .view(torch.bfloat16))
+        group.run()
+        got = yflat.clone()
+        yflat.fill_(float("nan"))
+        rabit.rabit_gemv_grouped(tup, workspace=group.workspace)
+        torch.cuda.synchronize()
+        assert torch.equal(got, yflat)
+        yo = 0
+        for i, (x, (N, K)) in enumerate(zip(xs, shapes)):
+            W = inputs.weight(7300 + i, N, K)
+            a, b = inputs.scales(7300 + i, W)
+            ref = oracle.layer(oracle.derive_signs(W, a, b), a, b, x)
+            assert normwise(got[yo:yo + N].cpu().numpy()[None, :], ref) <= TOL[torch.bfloat16]
+            yo += N
