@@ -152,25 +152,38 @@ scale_grads_tile_kernel(const float *__restrict__ G, int ldg, const uint32_t *__
     }
 }
 
-// The same pass with G staged by TMA, persistent: one CTA per SM walks its share of the
-// tiles (256 rows x 256 columns, eight boxes of 32 rows), and a producer warp keeps kStages
-// stages in flight across tile boundaries, so the stream never drains between tiles.  A stage
-// holds one box of G (32 rows x 256 columns, 32 KiB of fp32), the sign words of the same rows
-// and columns and the rows' a, all brought by TMA, so the consumers read shared memory only.
-// Eight consumer warps take four rows of each box; at a tile's end they add their column
-// sums in shared memory, in a fixed order.  Every wait is
-// bounded: an expired wait sets a fault bit and a flag in shared memory, the consumers stop
-// together at the end of the tile, and the producer lets its issued copies land before exiting.
+// The same pass with G staged by TMA, persistent and balanced to the box: the boxes (32 rows x
+// 256 columns of G), in column-tile-major order, are dealt as equal contiguous ranges to one
+// CTA per SM ("stream-K"), so no CTA has more than one box above the average.  A range spans
+// at most two column tiles (the host checks), so a CTA makes at most two runs.  A producer
+// warp keeps kStages stages in flight across run boundaries.  A stage holds one box of G
+// (32 KiB of fp32), the sign words of the same rows and columns and the rows' a, all brought
+// by TMA, so the consumers read shared memory only.  Eight consumer warps take four rows of
+// each box; row sums land in the (column tile, row) slot, which exactly one CTA writes; at a
+// run's end the warps add their column sums in shared memory, in a fixed order, into the
+// CTA's slot for that run (0 or 1), and pass 2 adds the slots of the CTAs that cover a column
+// tile in CTA order.  Every wait is bounded: an expired wait sets a fault bit and a flag in
+// shared memory, the consumers stop together at the end of the run, and the producer lets
+// its issued copies land before exiting.
 constexpr int kBoxRows = 32;
 constexpr int kBoxCols = 256;
 constexpr int kBoxBytes = kBoxRows * kBoxCols * 4;
 constexpr int kStages = 5;
-constexpr int kBoxesPerTile = 8;                 // 256 rows
 constexpr int kTmaThreads = 288;                 // 8 consumer warps + 1 producer warp
+constexpr int kMaxGrid = 160;                                 // CTAs of the stream-K pass, at most
 constexpr int kWordsBytesMax = kBoxRows * 32 * 4;             // sign words of a box (P = 3: 32 words a row)
 constexpr int kABytes = 1024;                                 // a of a box's rows (P x 32 floats), padded
 constexpr int kStageBytes = kBoxBytes + kWordsBytesMax + kABytes;
 constexpr int kTmaSmem = kStages * kStageBytes + 128;
+
+// First box of CTA c's range, and the CTA whose range holds box u (U boxes over G CTAs).
+__host__ __device__ inline int64_t sk_begin(int c, int64_t U, int G) { return U * c / G; }
+__host__ __device__ inline int sk_owner(int64_t u, int64_t U, int G) {
+    int c = static_cast<int>(u * G / U);
+    while (c + 1 < G && sk_begin(c + 1, U, G) <= u) ++c;
+    while (c > 0 && sk_begin(c, U, G) > u) --c;
+    return c;
+}
 
 template <int kP>
 __global__ void __launch_bounds__(kTmaThreads, 1)
@@ -198,8 +211,9 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nct = (K + kBoxCols - 1) / kBoxCols;
-    const int nrb = (N + kBoxRows * kBoxesPerTile - 1) / (kBoxRows * kBoxesPerTile);
-    const int ntiles = nct * nrb;
+    const int bpc = (N + kBoxRows - 1) / kBoxRows;             // boxes per column tile
+    const int64_t U = static_cast<int64_t>(nct) * bpc;
+    const int64_t u_begin = sk_begin(blockIdx.x, U, gridDim.x), u_end = sk_begin(blockIdx.x + 1, U, gridDim.x);
     int abort_flag = 0;
 
     if (threadIdx.x == 0) {
@@ -224,11 +238,9 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
             uint32_t last_parity[kStages] = {};
             bool ok = true;
             int q = 0;                                 // boxes of this CTA so far (ring position)
-            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-                const int ct = t % nct, rb = t / nct;
-                const int row0 = rb * kBoxRows * kBoxesPerTile;
-                const int boxes = min(kBoxesPerTile, (N - row0 + kBoxRows - 1) / kBoxRows);
-                for (int c = 0; c < boxes; ++c, ++q) {
+            for (int64_t u = u_begin; ok && u < u_end; ++u, ++q) {
+                const int ct = static_cast<int>(u / bpc), box = static_cast<int>(u % bpc);
+                {
                     const int s = q % kStages;
                     const uint32_t par = static_cast<uint32_t>(q / kStages) & 1u;
                     if (!mbar_wait_bounded(smem_u32(&empty[s]), par ^ 1u, &abort_flag, timeout_ns, fault,
@@ -239,9 +251,9 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
                     if ((debug & 1) && q == 0) continue;   // fault injection: this box never comes
                     const uint32_t bar = smem_u32(&full[s]);
                     mbar_arrive_expect_tx(bar, kTx);
-                    tma_load_2d(smem_u32(stage_g(s)), &tmap_g, bar, ct * kBoxCols, row0 + c * kBoxRows);
-                    tma_load_2d(smem_u32(stage_w(s)), &tmap_w, bar, ct * kRowWords, row0 + c * kBoxRows);
-                    tma_load_2d(smem_u32(stage_a(s)), &tmap_a, bar, row0 + c * kBoxRows, 0);
+                    tma_load_2d(smem_u32(stage_g(s)), &tmap_g, bar, ct * kBoxCols, box * kBoxRows);
+                    tma_load_2d(smem_u32(stage_w(s)), &tmap_w, bar, ct * kRowWords, box * kBoxRows);
+                    tma_load_2d(smem_u32(stage_a(s)), &tmap_a, bar, box * kBoxRows, 0);
                     issued[s] = true;
                     last_parity[s] = par;
                 }
@@ -262,11 +274,11 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
     // lane's columns: c0 + 128 st + 4 lane + t; group c0/32 + 4 st + lane/8, bits 4(lane%8) + t
     const uint32_t sh = 4 * (lane & 7);
     int q = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const int ct = t % nct, rb = t / nct;
+    int64_t u = u_begin;
+    for (int side = 0; u < u_end; ++side) {       // a run: this CTA's boxes of one column tile
+        const int ct = static_cast<int>(u / bpc);
+        const int64_t run_end = min(u_end, static_cast<int64_t>(ct + 1) * bpc);
         const int c0 = ct * kBoxCols;
-        const int row0 = rb * kBoxRows * kBoxesPerTile;
-        const int boxes = min(kBoxesPerTile, (N - row0 + kBoxRows - 1) / kBoxRows);
         float bcol[kP][kSteps][4], cacc[kP][kSteps][4];
 #pragma unroll
         for (int st = 0; st < kSteps; ++st)
@@ -279,13 +291,14 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
                     cacc[k][st][tt] = 0.0f;
                 }
             }
-        for (int c = 0; c < boxes; ++c, ++q) {
+        for (; u < run_end; ++u, ++q) {
+            const int row0 = static_cast<int>(u % bpc) * kBoxRows;
             const int s = q % kStages;
             const bool ok = mbar_wait_bounded(smem_u32(&full[s]), static_cast<uint32_t>(q / kStages) & 1u,
                                               &abort_flag, timeout_ns, fault, FAULT_SCALE_GRADS_WAIT);
             // An expired wait ends this warp's boxes: it stops releasing stages, so the producer's
             // own bounded wait expires and it drains the copies it issued before the CTA exits;
-            // the flag stops every consumer warp at the end of this tile.
+            // the flag stops every consumer warp at the end of this run.
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) s_abort = 1;
                 break;
@@ -296,7 +309,7 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
 #pragma unroll
             for (int i = 0; i < kRowsPerWarp; ++i) {
                 const int r = warp * kRowsPerWarp + i;
-                const int n = row0 + c * kBoxRows + r;
+                const int n = row0 + r;
                 float racc[kP], av[kP];
                 uint32_t wv[kSteps][kP];
 #pragma unroll
@@ -341,15 +354,13 @@ scale_grads_tma_kernel(const __grid_constant__ CUtensorMap tmap_g, const __grid_
 #pragma unroll
                 for (int tt = 0; tt < 4; ++tt) colsum[warp][k][128 * st + 4 * lane + tt] = cacc[k][st][tt];
         asm volatile("bar.sync 1, 256;" ::: "memory");   // the 8 consumer warps only
-        for (int u = threadIdx.x; u < kP * kBoxCols; u += 256) {
-            const int k = u / kBoxCols, cc = u % kBoxCols;
-            const int j = c0 + cc;
-            if (j >= K) continue;
+        for (int e = threadIdx.x; e < kP * kBoxCols; e += 256) {
+            const int k = e / kBoxCols, cc = e % kBoxCols;
             float v = 0.0f;
             for (int w = 0; w < 8; ++w) v += colsum[w][k][cc];
-            ws_b[(static_cast<int64_t>(k) * nrb + rb) * K + j] = v;
+            ws_b[((static_cast<int64_t>(k) * gridDim.x + blockIdx.x) * 2 + side) * kBoxCols + cc] = v;
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");   // colsum is rewritten by the next tile
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // colsum is rewritten by the next run
         if (s_abort) break;                              // every consumer warp sees the same flag here
     }
 }
@@ -368,9 +379,12 @@ __device__ __forceinline__ float strided_sum(const float *__restrict__ p, int co
     return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
+// sk_grid > 0: ws_b holds the stream-K pass's run slots [P][sk_grid][2][kBoxCols]; otherwise the
+// tile pass's row-block slots [P][nrb][K].
 __global__ void __launch_bounds__(256)
 scale_grads_sum_kernel(const float *__restrict__ ws_a, const float *__restrict__ ws_b, int N, int K,
-                       int P, int nct, int nrb, float *__restrict__ grad_a, float *__restrict__ grad_b) {
+                       int P, int nct, int nrb, int sk_grid, float *__restrict__ grad_a,
+                       float *__restrict__ grad_b) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     const int64_t na = static_cast<int64_t>(P) * N, nb = static_cast<int64_t>(P) * K;
@@ -379,6 +393,20 @@ scale_grads_sum_kernel(const float *__restrict__ ws_a, const float *__restrict__
         if (t < na) {
             const int64_t k = t / N, n = t % N;
             grad_a[t] = strided_sum(ws_a + k * nct * N + n, nct, N);
+        } else if (sk_grid > 0) {
+            // the CTAs whose ranges cover column tile ct, in CTA order; the first one's slot is
+            // 1 when its range began in an earlier tile
+            const int64_t u = t - na, k = u / K, j = u % K;
+            const int ct = static_cast<int>(j / kBoxCols), cc = static_cast<int>(j % kBoxCols);
+            const int bpc = (N + kBoxRows - 1) / kBoxRows;
+            const int64_t U = static_cast<int64_t>(nct) * bpc, ub = static_cast<int64_t>(ct) * bpc;
+            const int cf = sk_owner(ub, U, sk_grid), cl = sk_owner(ub + bpc - 1, U, sk_grid);
+            float v = 0.0f;
+            for (int c = cf; c <= cl; ++c) {
+                const int side = (c == cf && sk_begin(c, U, sk_grid) < ub) ? 1 : 0;
+                v += __ldg(ws_b + ((k * sk_grid + c) * 2 + side) * kBoxCols + cc);
+            }
+            grad_b[u] = v;
         } else {
             const int64_t u = t - na, k = u / K, j = u % K;
             grad_b[u] = strided_sum(ws_b + k * nrb * K + j, nrb, K);
@@ -388,10 +416,13 @@ scale_grads_sum_kernel(const float *__restrict__ ws_a, const float *__restrict__
 
 }  // namespace
 
+// [P][nct][N] row-sum slots, then the column-sum slots: the tile pass's [P][nrb][K] or the
+// stream-K pass's [P][kMaxGrid][2][kBoxCols], whichever is larger.
 size_t scale_grads_workspace_bytes(int N, int K, int P) {
     const size_t nct = (static_cast<size_t>(K) + tile_cols(P) - 1) / tile_cols(P);
     const size_t nrb = (static_cast<size_t>(N) + kTileRows - 1) / kTileRows;
-    return static_cast<size_t>(P) * (nct * N + nrb * K) * sizeof(float);
+    const size_t colslots = std::max(nrb * K, static_cast<size_t>(kMaxGrid) * 2 * kBoxCols);
+    return static_cast<size_t>(P) * (nct * N + colslots) * sizeof(float);
 }
 
 cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, const uint32_t *packed,
@@ -416,8 +447,13 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
     // TMA-staged pass when tensor maps can describe G (16-byte aligned base and pitch) and a.
     auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
     // (a is staged by TMA as well: 16-byte aligned base and rows of N floats, N a multiple of 4)
+    // The stream-K deal: a CTA's range of boxes may touch at most two column tiles.
+    const int bpc = (N + kBoxRows - 1) / kBoxRows;
+    const int64_t boxes = static_cast<int64_t>(nct) * bpc;
+    const int sk_grid = static_cast<int>(std::min<int64_t>({boxes, static_cast<int64_t>(ctx.num_sms), kMaxGrid}));
+    const bool two_runs = (boxes + sk_grid - 1) / sk_grid - 1 <= bpc;
     const bool tma = encode && (reinterpret_cast<uintptr_t>(G) % 16 == 0) && ((static_cast<int64_t>(ldg) * 4) % 16 == 0) &&
-                     (reinterpret_cast<uintptr_t>(a) % 16 == 0) && (N % 4 == 0);
+                     (reinterpret_cast<uintptr_t>(a) % 16 == 0) && (N % 4 == 0) && two_runs;
     if (tma) {
         CUtensorMap tmap;
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
@@ -450,8 +486,7 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
                      uint32_t *, uint64_t, int) = P == 2 ? scale_grads_tma_kernel<2> : scale_grads_tma_kernel<3>;
         e = ensure_smem_optin(ctx, kern, kTmaSmem, opted[P - 2]);
         if (e != cudaSuccess) return e;
-        nrb = (N + kBoxRows * kBoxesPerTile - 1) / (kBoxRows * kBoxesPerTile);
-        cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(nct) * nrb, ctx.num_sms)));
+        cfg.gridDim = dim3(static_cast<unsigned>(sk_grid));
         cfg.blockDim = dim3(kTmaThreads);
         cfg.dynamicSmemBytes = kTmaSmem;
         e = cudaLaunchKernelEx(&cfg, kern, tmap, tmap_w, tmap_a, b, N, K, Wr, ws_a, ws_b, fault_word, timeout_ns,
@@ -468,7 +503,8 @@ cudaError_t launch_scale_grads(const LaunchCtx &ctx, const float *G, int ldg, co
     cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(ctx.num_sms) * 8)));
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, scale_grads_sum_kernel, ws_a, ws_b, N, K, P, nct, nrb, grad_a, grad_b);
+    return cudaLaunchKernelEx(&cfg, scale_grads_sum_kernel, ws_a, ws_b, N, K, P, nct, nrb, tma ? sk_grid : 0,
+                              grad_a, grad_b);
 }
 
 }  // namespace rabit

@@ -135,7 +135,9 @@ def test_gemm_validation(lib):
 def test_scale_grads_validation(lib):
     f = lib.rabit_scale_grads
     need = lib.rabit_scale_grads_workspace_bytes(8, 16, 2)
-    assert need == 2 * (1 * 8 + 1 * 16) * 4          # one column tile, one row block
+    # row sums: one column tile x 8 rows; column sums: the larger of one row block x 16
+    # columns (tile pass) and 160 CTAs x 2 runs x 256 columns (stream-K pass)
+    assert need == 2 * (1 * 8 + max(1 * 16, 160 * 2 * 256)) * 4
     args = lambda **kw: [P(kw.get("G", FAKE)), kw.get("ldg", 16), P(kw.get("packed", FAKE)), P(FAKE), P(FAKE),
                          kw.get("N", 8), kw.get("K", 16), kw.get("P", 2), P(FAKE), P(FAKE),
                          P(kw.get("ws", FAKE)), kw.get("wsb", need), None]
