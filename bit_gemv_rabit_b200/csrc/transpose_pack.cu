@@ -11,8 +11,10 @@
 // A CTA transposes a tile of 256 rows x 256 columns of every plane.  The tile's words come
 // into shared memory with coalesced loads (8 groups x G words of each input row, in a row
 // padded by one word so column reads are free of bank conflicts), each warp turns 32 x 32-bit
-// blocks around with 32 ballots (lane l holds input row l's word; the ballot of bit b is
-// output row b's word), and the transposed tile leaves with coalesced stores.
+// blocks around (lane l holds input row l's word and ends with output row l's), and the
+// transposed tile leaves with coalesced stores.  The block transpose is the recursive one:
+// for j = 16, 8, 4, 2, 1, lanes l and l ^ j exchange words and swap the off-diagonal j x j
+// sub-blocks of every 2j x 2j block (five shuffles instead of 32 ballots).
 #include <cstdint>
 
 #include "rabit_device.cuh"
@@ -49,11 +51,16 @@ transpose_pack_kernel(const uint32_t *__restrict__ in, int N, int K, int wr_in, 
         const int k = t % G, blk = t / G, bi = blk / kTileGroups, bj = blk - bi * kTileGroups;
         uint32_t mine = 0u;
         if (k < P) {                                   // (the padding word of a group stays 0)
-            const uint32_t w = tin[(32 * bi + lane) * kRow + bj * G + k];
+            mine = tin[(32 * bi + lane) * kRow + bj * G + k];
+            // bit c of row r -> bit r of row c.  low: the columns c with (c & j) == 0.
+            constexpr uint32_t kLow[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
 #pragma unroll
-            for (int b = 0; b < 32; ++b) {
-                const uint32_t col = __ballot_sync(0xffffffffu, (w >> b) & 1u);
-                if (lane == b) mine = col;
+            for (int step = 0; step < 5; ++step) {
+                const int j = 16 >> step;
+                const uint32_t low = kLow[step], high = ~low;
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, j);
+                mine = (lane & j) ? (((other & high) >> j) | (mine & high))     // lower row of the pair
+                                  : ((mine & low) | ((other & low) << j));      // upper row of the pair
             }
         }
         // output row j0 + 32 bj + lane, output group n0 / 32 + bi, path k
