@@ -28,7 +28,10 @@ def normwise(y, ref):
     return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-300))
 
 
-@pytest.mark.parametrize("N,K,P", [(33, 129, 2), (300, 520, 2), (1024, 4096, 2), (200, 1100, 3), (4096, 4096, 3)])
+# (64, 40000, 3): a CTA's range of boxes spans two column tiles of a one-or-two-box column;
+# (32, 80000, 2): ranges would span three column tiles, so the direct-load pass runs
+@pytest.mark.parametrize("N,K,P", [(33, 129, 2), (300, 520, 2), (1024, 4096, 2), (200, 1100, 3), (4096, 4096, 3),
+                                   (64, 40000, 3), (32, 80000, 2)])
 def test_scale_grads_match_oracle(N, K, P):
     seed = 500 + N + P
     W = inputs.weight(seed, N, K)
