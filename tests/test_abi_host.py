@@ -256,3 +256,22 @@ def test_gemm_grouped_validation(lib):
     assert f(arr(), 2, 4, 8, P(FAKE), need, None) == UNSUP
     assert f(arr(), 2, 2, 8, P(FAKE), need - 1, None) == WS
     assert f(arr(), 2, 2, 8, P(FAKE + 128), need, None) == ALIGN
+
+
+def test_prepared_gemv_group_marshals_the_plain_call(lib):
+    """GemvGroup builds the same layer array as the plain grouped call, keeps its tensors,
+    and sizes the workspace with rabit_gemv_grouped_workspace_bytes (no launch here)."""
+    layers = []
+    for N, K in ((64, 256), (130, 520)):
+        x = torch.zeros((3, K), dtype=torch.bfloat16)
+        y = torch.zeros((3, N), dtype=torch.float32)
+        layers.append((torch.zeros(rabit.rabit_packed_words(N, K, 2), dtype=torch.int32).view(torch.uint32),
+                       torch.ones((2, N)), torch.ones((2, K)), N, K, x, y))
+    group = rabit.GemvGroup(layers)
+    want = rabit._layer_array(layers)
+    for got, ref in zip(group._arr, want):
+        for field, _ in rabit.GemvLayer._fields_:
+            assert getattr(got, field) == getattr(ref, field)
+    assert group._scalars == (2, 2, rabit.RABIT_BF16, 3)
+    assert group.workspace.numel() == rabit.rabit_gemv_grouped_workspace_bytes(layers) > 0
+    assert group.layers[0][5] is layers[0][5]
